@@ -1,0 +1,120 @@
+"""Planted mistakes: each plausible slip in the oracle must fail a pin.
+
+Every case edits a copy of oracle/split12_oracle.c (the committed oracle is
+never touched), compiles it with gcc into a temporary directory, binds it and
+runs a quick battery of the same pins as test_oracle_pins.py.  A mutant that
+passes the battery would mean the pins cannot see that mistake.
+"""
+import os
+
+import numpy as np
+import pytest
+
+from conftest import golden_expected_bytes, golden_two_tiles_weights, load_golden
+from decode_split12_b200 import workloads as wl
+from oracle import build_oracle
+from oracle.oracle import Oracle, load
+
+SRC = build_oracle.SRC
+
+MUTANTS = {
+    "window_14_wide": [("e <= b + ORACLE_WINDOW - 1", "e <= b + ORACLE_WINDOW - 2")],
+    "ties_to_largest_base": [("if (!have || c > best_count)", "if (!have || c >= best_count)")],
+    "base_241_excluded": [("for (uint32_t b = 0; b <= ORACLE_MAX_BASE; b++)",
+                           "for (uint32_t b = 0; b < ORACLE_MAX_BASE; b++)")],
+    "nibbles_swapped_consistently": [
+        ("code[pos / 2] = (uint8_t)c;", "code[pos / 2] = (uint8_t)(c << 4);"),
+        ("code[pos / 2] |= (uint8_t)(c << 4);", "code[pos / 2] |= (uint8_t)c;"),
+        ("return (pos % 2 == 0) ? (byte & 0x0Fu) : (uint32_t)(byte >> 4);",
+         "return (pos % 2 == 1) ? (byte & 0x0Fu) : (uint32_t)(byte >> 4);"),
+    ],
+    "sign_dropped_from_raw": [("(oracle_bf16_sign(v) << 7)", "(0u << 7)")],
+    "mantissa_mask_6_bits": [("return w & 0x7Fu; }", "return w & 0x3Fu; }")],
+    "decode_exponent_off_by_one": [("uint32_t e = b + c;", "uint32_t e = b + c + 1;")],
+    "decode_sign_wrong_bit": [("((uint32_t)(r & 0x80) << 8)", "((uint32_t)(r & 0x80) << 7)")],
+    "escapes_read_backwards": [("get_u16(V->esc + 2 * (uint64_t)(lo + k))",
+                                "get_u16(V->esc + 2 * (uint64_t)(hi - 1 - k))")],
+    "escape_count_check_dropped": [("if (lo + k != hi) return ORACLE_ERR_CORRUPT;", "")],
+    "magnitude_without_abs": [("mag += fabs(p);", "mag += p;")],
+    "weight_operand_transposed": [("oracle_bf16_to_double(w[n * cols + k])",
+                                   "oracle_bf16_to_double(w[k * rows + n])")],
+    "bf16_widened_by_15": [("uint32_t bits = (uint32_t)w << 16;", "uint32_t bits = (uint32_t)w << 15;")],
+    "last_plane_unpadded": [("L->total = L->off_esc + pad_to_align(2 * n_esc);",
+                             "L->total = L->off_esc + 2 * n_esc;")],
+    "entropy_in_nats": [("h -= p * log2(p);", "h -= p * log(p);")],
+    "escape_stored_byte_swapped": [("esc[2 * written] = (uint8_t)(v & 0xFF);\n                esc[2 * written + 1] = (uint8_t)(v >> 8);",
+                                    "esc[2 * written] = (uint8_t)(v >> 8);\n                esc[2 * written + 1] = (uint8_t)(v & 0xFF);")],
+}
+
+
+def _battery(o: Oracle):
+    """Raises AssertionError (or an oracle error) when any pin fails."""
+    d = load_golden("two_tiles.json")
+    w = golden_two_tiles_weights(d)
+    blob = o.encode(w)
+    assert blob.size == d["total_bytes"]
+    assert np.array_equal(blob, golden_expected_bytes(d))
+    # exhaustive round trips
+    allp = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    for p in (allp, allp[wl.rng_for(0, 1).permutation(allp.size)]):
+        wt = p.reshape(512, 128)
+        b2 = o.encode(wt)
+        assert np.array_equal(o.decode(b2), wt)
+    assert o.stats(o.encode(allp.reshape(512, 128)))["n_esc"] == 0
+    # brute-force bases
+    for seed in range(12):
+        tile = wl.rng_for(seed, 3).integers(0, 1 << 16, size=128).astype(np.uint16)
+        e = (tile.astype(np.int64) >> 7) & 0xFF
+        counts = [int(np.sum((e < b) | (e > b + 14))) for b in range(242)]
+        b, n = o.tile_base(tile)
+        assert n == min(counts) and b == counts.index(min(counts))
+    # exact escape count of the stress recipe
+    ws, planted = wl.escape_stress(0.02, seed=0, rows=64, cols=1024)
+    assert o.stats(o.encode(ws))["n_esc"] == planted
+    # products: one-hot column, integer sums, magnitudes
+    wn = wl.normal_with_outliers(33, 384, 0.02, 0.01, 3)
+    bn = o.encode(wn)
+    x = np.zeros((1, 384), np.uint16)
+    x[0, 200] = 0x3F80
+    y, s = o.gemv_f64(bn, x)
+    col = wl.bf16_bits_to_f32(wn[:, 200]).astype(np.float64)
+    assert np.array_equal(y[0], col) and np.array_equal(s[0], np.abs(col))
+    vals = wl.rng_for(9, 0).integers(-8, 9, size=(20, 256)).astype(np.float32)
+    bi = o.encode(wl.to_bf16_bits(vals))
+    y, s = o.gemv_f64(bi, np.full((1, 256), 0x3F80, np.uint16))
+    assert np.array_equal(y[0], vals.sum(1)) and np.array_equal(s[0], np.abs(vals).sum(1))
+    # entropy near the pages' ~2.6 bits
+    st = o.stats(o.encode(wl.normal_with_outliers(64, 2048, 0.02, 0.0, 0)))
+    assert 2.4 <= st["exp_entropy_bits"] <= 2.8
+    # corruption: a flipped code nibble must be refused
+    wc = wl.normal_with_outliers(8, 512, 0.02, 0.01, 4)
+    bc = o.encode(wc)
+    code = bc[256 + 4096: 256 + 4096 + 2048]
+    k = int(np.nonzero((code & 0x0F) != 0x0F)[0][0])
+    bc[256 + 4096 + k] |= 0x0F
+    assert o.decode_rc(bc) != 0
+    # ... and so must an escape code turned into an ordinary one
+    bc = o.encode(wc)
+    code = bc[256 + 4096: 256 + 4096 + 2048]
+    k = int(np.nonzero((code & 0x0F) == 0x0F)[0][0])
+    bc[256 + 4096 + k] &= 0xF0
+    assert o.decode_rc(bc) != 0
+
+
+def test_unmutated_oracle_passes_battery(oracle):
+    _battery(oracle)
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_is_caught(name, tmp_path):
+    src = open(SRC).read()
+    for old, new in MUTANTS[name]:
+        assert src.count(old) == 1, f"mutation anchor not unique/missing: {old!r}"
+        src = src.replace(old, new)
+    path = tmp_path / "mutant.c"
+    path.write_text(src)
+    lib = build_oracle.build(str(path), str(tmp_path / f"lib_{name}.so"), extra=("-w",))
+    o = Oracle(load(lib))
+    with pytest.raises(Exception):
+        _battery(o)
+    assert os.path.exists(lib)
