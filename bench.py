@@ -1,0 +1,528 @@
+#!/usr/bin/env python
+"""Benchmark of the Split12 fused decode-GEMV (and the other kernels).
+
+Default workload (one JSON line on rank 0): one Llama-style 8B decoder layer
+-- q, o 4096x4096; k, v 1024x4096; gate, up 14336x4096; down 4096x14336,
+Student-t(5) weights scaled to std 1/sqrt(in) -- encoded once into Split12
+containers resident in HBM.  A step is the seven fused decode-GEMVs of the
+layer at batch 1 (the decode phase of one token).  The metric is effective
+BF16 GB/s = 2 bytes x weights / time, with the fraction of the measured HBM
+copy bandwidth achieved on the compressed bytes actually moved.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+                    [--workload llama8b|single|escape|mlp70b|stack]
+
+Several GPUs run independent replicas (the path does not shard): every
+rank times its own copy and rank 0 reports the sum of work over the max
+time over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from decode_split12_b200 import workloads as wl  # noqa: E402
+
+HBM_FALLBACK_GBS = 6650.0
+L2_BYTES_B200 = 126 * 1024 * 1024
+METRIC = "fused decode-GEMV effective BF16 GB/s & % HBM roofline on compressed bytes"
+
+
+# --------------------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d.get("bf16_tflops", 1590.0)), \
+            float(d.get("bf16_tflops_sustained", 1400.0)), "measured"
+    except Exception:
+        return HBM_FALLBACK_GBS, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.period = period_s
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thr = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = device_index
+            if vis:
+                parts = [p for p in vis.split(",") if p.strip()]
+                if device_index < len(parts) and parts[device_index].strip().isdigit():
+                    idx = int(parts[device_index])
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                try:
+                    reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except Exception:
+                    reasons = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.samples.append((mhz, int(reasons)))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thr:
+            self._thr.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = [s[0] for s in self.samples]
+        bits = 0
+        for _, r in self.samples:
+            bits |= r
+        reasons = [name for b, name in self.REASONS.items() if bits & b and name != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(mhz)), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(mhz)}
+
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        backend = os.environ.get("S12_BENCH_BACKEND", "nccl")
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value: float, world: int) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def dev16(a: np.ndarray):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint16).view(np.int16)).cuda()
+
+
+def time_graph(graph, steps: int, world: int, sampler=None):
+    """Replays `graph` `steps` times between two events on the current
+    stream, bracketed by a barrier and synchronisations; returns seconds
+    (max over ranks)."""
+    import torch
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    ctx = sampler if sampler is not None else _Null()
+    with ctx:
+        start.record()
+        for _ in range(steps):
+            graph.replay()
+        end.record()
+        torch.cuda.synchronize()
+    barrier(world)
+    sec = start.elapsed_time(end) / 1e3
+    return max_over_ranks(sec, world)
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def capture(fn):
+    import torch
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()  # first run outside capture (sets kernel attributes)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def prewarm(graph, seconds: float = 0.3):
+    """Untimed replays so clocks are at their working level."""
+    import torch
+    t0 = time.time()
+    while time.time() - t0 < seconds:
+        for _ in range(20):
+            graph.replay()
+        torch.cuda.synchronize()
+
+
+def load_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch recorded from an ncu capture (profiles/), used
+    only if the kernel source has not changed since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d[kernel][workload]
+        import hashlib
+        src = os.path.join(ROOT, "decode_split12_b200", "csrc", e["source"])
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if h != e["source_sha256_16"]:
+            return None
+        return e
+    except Exception:
+        return None
+
+
+# --------------------------------------------------------------------------- llama8b (default)
+
+class Llama8bLayer:
+    def __init__(self, batch: int, seed: int = 0, need_bf16: bool = True):
+        import torch
+
+        from decode_split12_b200 import s12
+        self.s12 = s12
+        self.batch = batch
+        mats, xs = wl.llama8b_layer(seed, batch)
+        self.names = list(wl.LLAMA8B_SHAPES)
+        self.weights = sum(r * c for r, c in wl.LLAMA8B_SHAPES.values())
+        self.containers, self.views, self.x, self.y = {}, {}, {}, {}
+        self.host_blobs = {}
+        self.w_dev = {}
+        self.x_host = {}
+        for n in self.names:
+            wd = dev16(mats[n])
+            blob = s12.s12_encode(wd)
+            self.containers[n] = blob
+            self.views[n] = s12.s12_open(blob)
+            if need_bf16:
+                self.w_dev[n] = wd
+            else:
+                del wd
+            self.x[n] = dev16(xs[n])
+            self.x_host[n] = xs[n]
+            self.y[n] = torch.empty((batch, mats[n].shape[0]), dtype=torch.float32, device="cuda")
+        self.mats = mats
+        torch.cuda.synchronize()
+        self.compressed = sum(int(v.container_bytes) for v in self.views.values())
+        self.read_bytes = sum(self._alg_bytes(n) for n in self.names)
+
+    def _alg_bytes(self, n):
+        v = self.views[n]
+        r, c = int(v.rows), int(v.cols)
+        # every plane is read once (payload, per-tile base + offsets, escapes),
+        # x is read, y is written
+        return (r * c * 3 // 2 + int(v.n_tiles) * 5 + 4 + 2 * int(v.n_esc) + self.batch * c * 2 +
+                self.batch * r * 4)
+
+    def set_batch_x(self, batch, seed=0):
+        import torch
+        self.batch = batch
+        for i, n in enumerate(self.names):
+            c = wl.LLAMA8B_SHAPES[n][1]
+            xs = wl.activations(batch, c, seed, 1000 + i)
+            self.x[n] = dev16(xs)
+            self.x_host[n] = xs
+            self.y[n] = torch.empty((batch, wl.LLAMA8B_SHAPES[n][0]), dtype=torch.float32, device="cuda")
+        self.read_bytes = sum(self._alg_bytes(n) for n in self.names)
+
+    def step(self):
+        for n in self.names:
+            self.s12.s12_gemv(self.views[n], self.x[n], self.y[n])
+
+    def step_bf16_own(self):
+        for n in self.names:
+            self.s12.s12_bf16_gemv(self.w_dev[n], self.x[n], self.y[n])
+
+    def step_bf16_torch(self):
+        import torch
+        for n in self.names:
+            torch.nn.functional.linear(self.x[n].view(torch.bfloat16), self.w_dev[n].view(torch.bfloat16))
+
+
+def e2e_llama(layer: Llama8bLayer, steps: int, warmup: int, world: int):
+    """Same metric through the public API with host buffers: each step copies
+    every matrix's x from pinned host memory, runs the seven GEMVs and copies
+    every y back to pinned host memory."""
+    import torch
+    xh = {n: torch.from_numpy(layer.x_host[n].view(np.int16)).pin_memory() for n in layer.names}
+    yh = {n: torch.empty(tuple(layer.y[n].shape), dtype=torch.float32).pin_memory() for n in layer.names}
+    h2d = sum(xh[n].numel() * 2 for n in layer.names)
+    d2h = sum(yh[n].numel() * 4 for n in layer.names)
+
+    def step():
+        for n in layer.names:
+            layer.x[n].copy_(xh[n], non_blocking=True)
+        layer.step()
+        for n in layer.names:
+            yh[n].copy_(layer.y[n], non_blocking=True)
+
+    g = capture(step)
+    for _ in range(max(warmup, 3)):
+        g.replay()
+    torch.cuda.synchronize()
+    sec = time_graph(g, steps, world)
+    return sec / steps, h2d, d2h, g
+
+
+def cpu_baseline_llama(target_s: float = 12.0):
+    """The oracle as it stands (single-threaded C, FP64) on a bounded sample:
+    a fraction of the rows of each of the seven matrices, B = 1, scaled so the
+    timed oracle work takes about `target_s` seconds."""
+    from oracle.oracle import Oracle
+    orc = Oracle()
+    mats, xs = wl.llama8b_layer(0, 1)
+    g = wl.rng_for(99, 0)
+
+    def run(frac):
+        weights, secs = 0, 0.0
+        for n in wl.LLAMA8B_SHAPES:
+            r, c = wl.LLAMA8B_SHAPES[n]
+            k = max(1, int(round(frac * r)))
+            rows = np.sort(g.choice(r, k, replace=False))
+            blob = orc.encode(mats[n][rows])
+            t0 = time.perf_counter()
+            orc.gemv_f64(blob, xs[n])
+            secs += time.perf_counter() - t0
+            weights += k * c
+        return weights, secs
+
+    w1, s1 = run(0.002)
+    frac = min(1.0, 0.002 * target_s / max(s1, 1e-6))
+    weights, secs = run(frac)
+    return {"value": round(2 * weights / secs / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{frac * 100:.2f}% of the rows of each of the 7 matrices (decode + FP64 GEMV, B=1), "
+                      f"{weights} weights in {secs:.1f} s on 1 of {os.cpu_count()} host cores"}
+
+
+def run_llama8b(args, world, rank):
+    import torch
+    hbm, _, _, peak_kind = load_peaks()
+    layer = Llama8bLayer(args.batch)
+    g = capture(layer.step)
+    for _ in range(max(args.warmup, 3)):
+        g.replay()
+    torch.cuda.synchronize()
+    prewarm(g)
+    sampler = ClockSampler(torch.cuda.current_device())
+    sec = time_graph(g, args.steps, world, sampler)
+    ms = sec / args.steps * 1e3
+    t_step = sec / args.steps
+    value_rank = 2 * layer.weights / t_step / 1e9
+    value = value_rank * world  # all ranks processed the same amount; time is the max
+    achieved = layer.read_bytes / t_step / 1e9
+    extra = {}
+    # batch 4 and 8 on the same containers
+    for b in (4, 8):
+        if b == args.batch:
+            continue
+        layer.set_batch_x(b)
+        gb = capture(layer.step)
+        for _ in range(3):
+            gb.replay()
+        sb = time_graph(gb, max(20, args.steps // 4), world) / max(20, args.steps // 4)
+        extra[f"B{b}"] = {"us_per_layer": round(sb * 1e6, 2), "effective_bf16_GBs": round(2 * layer.weights / sb / 1e9, 1),
+                          "hbm_frac": round(layer.read_bytes / sb / 1e9 / hbm, 4)}
+        del gb
+    layer.set_batch_x(args.batch)
+    # uncompressed BF16 baselines at the same batch: own kernel and cuBLAS
+    for name, fn in (("bf16_own_gemv", layer.step_bf16_own), ("bf16_torch_linear", layer.step_bf16_torch)):
+        gb = capture(fn)
+        for _ in range(3):
+            gb.replay()
+        nb = max(20, args.steps // 2)
+        sb = time_graph(gb, nb, world) / nb
+        extra[name] = {"us_per_layer": round(sb * 1e6, 2), "GBs": round(2 * layer.weights / sb / 1e9, 1),
+                       "hbm_frac": round(2 * layer.weights / sb / 1e9 / hbm, 4)}
+        del gb
+    e2e_t, h2d, d2h, ge = e2e_llama(layer, max(20, args.steps // 2), args.warmup, world)
+    del ge
+    traffic = load_traffic("gemv_kernel", f"llama8b_b{args.batch}")
+    out = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": {
+            "workload": f"llama8b-layer decode GEMV, B={args.batch}: q,o 4096x4096; k,v 1024x4096; "
+                        f"gate,up 14336x4096; down 4096x14336 (Student-t(5)/sqrt(in), Split12 resident in HBM)",
+            "batch": args.batch,
+            "weights_per_step": layer.weights,
+            "compressed_bytes_per_step": layer.compressed,
+            "algorithmic_bytes_per_step": layer.read_bytes,
+            "launches_per_step": 7,
+            "l2": f"inputs larger than L2: {layer.compressed / 1e6:.1f} MB of containers per step vs "
+                  f"{L2_BYTES_B200 / 2**20:.0f} MiB L2",
+            "parallelism": "replicas" if world > 1 else "single GPU",
+        },
+        "roofline": {
+            "bound": "hbm",
+            "achieved": round(achieved, 1),
+            "peak": hbm,
+            "unit": "GB/s",
+            "frac": round(achieved / hbm, 4),
+            "traffic": (traffic or {}).get("dram_bytes_per_step"),
+            "peak_kind": peak_kind,
+            "kernel": "gemv_kernel",
+        },
+        "clocks": sampler.summary(),
+        "e2e": {"value": round(2 * layer.weights / e2e_t / 1e9 * world, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 7 * args.steps,
+        "extra": extra,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline_llama()
+    return out
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the CPU oracle, as it stands, on the same workload and
+    metric; each step is a bounded sample (1 % of the rows of each matrix)."""
+    if rank != 0:
+        return None
+    from oracle.oracle import Oracle
+    orc = Oracle()
+    mats, xs = wl.llama8b_layer(0, args.batch)
+    g = wl.rng_for(98, 0)
+    subs = {}
+    weights = 0
+    for n in wl.LLAMA8B_SHAPES:
+        r, c = wl.LLAMA8B_SHAPES[n]
+        k = max(1, int(round(0.01 * r)))
+        rows = np.sort(g.choice(r, k, replace=False))
+        subs[n] = orc.encode(mats[n][rows])
+        weights += k * c
+
+    def step():
+        for n in subs:
+            orc.gemv_f64(subs[n], xs[n])
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    sec = time.perf_counter() - t0
+    t_step = sec / args.steps
+    value = 2 * weights / t_step / 1e9
+    cb = {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+          "sample": f"1% of the rows of each of the 7 llama8b-layer matrices per step ({weights} weights), "
+                    f"B={args.batch}, decode + FP64 GEMV, 1 of {os.cpu_count()} host cores"}
+    return {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(t_step * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"llama8b-layer decode GEMV, B={args.batch} (oracle on a 1% row sample)",
+                       "batch": args.batch},
+            "impl": "reference", "cpu_baseline": cb,
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+
+
+# --------------------------------------------------------------------------- main
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["split12", "reference"], default="split12")
+    ap.add_argument("--workload", choices=["llama8b"], default="llama8b")
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_init()
+    if args.impl == "reference":
+        out = run_reference(args, world, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return 0
+    import torch
+    torch.cuda.set_device(local)
+    from decode_split12_b200 import s12
+    s12.device_check()
+    out = run_llama8b(args, world, rank)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,215 @@
+// s12_api.cu -- the C ABI of libs12.so (declared in include/s12.h): argument
+// checks, container parsing, and dispatch to the kernel launchers.
+#include <atomic>
+#include <cmath>
+#include <cstring>
+
+#include "s12_device.cuh"
+#include "s12_launch.h"
+
+namespace s12 {
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sms[kMaxDevices];
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3) == 0; }
+
+int check_view(const s12_view *v) {
+    if (!v || !v->container || !v->raw || !v->code || !v->base || !v->esc_off || !v->esc) return S12_ERR_ARG;
+    if (v->rows == 0 || v->cols == 0 || v->cols % kTile) return S12_ERR_SHAPE;
+    if (!aligned16(v->container)) return S12_ERR_ALIGN;
+    return S12_OK;
+}
+
+uint32_t get_u32(const uint8_t *p) {
+    return uint32_t(p[0]) | uint32_t(p[1]) << 8 | uint32_t(p[2]) << 16 | uint32_t(p[3]) << 24;
+}
+uint64_t get_u64(const uint8_t *p) { return uint64_t(get_u32(p)) | uint64_t(get_u32(p + 4)) << 32; }
+}  // namespace
+
+cudaError_t device_sms(int *sms) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < kMaxDevices) {
+        const int c = g_sms[dev].load(std::memory_order_relaxed);
+        if (c > 0) {
+            *sms = c;
+            return cudaSuccess;
+        }
+    }
+    int n = 0;
+    e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < kMaxDevices) g_sms[dev].store(n, std::memory_order_relaxed);
+    *sms = n;
+    return cudaSuccess;
+}
+
+}  // namespace s12
+
+using namespace s12;
+
+extern "C" {
+
+const char *s12_error_string(int status) {
+    switch (status) {
+        case S12_OK: return "S12_OK";
+        case S12_ERR_ARG: return "S12_ERR_ARG: null pointer or invalid size";
+        case S12_ERR_SHAPE: return "S12_ERR_SHAPE: unsupported shape or batch";
+        case S12_ERR_ALIGN: return "S12_ERR_ALIGN: device pointer not 16-byte aligned";
+        case S12_ERR_CAPACITY: return "S12_ERR_CAPACITY: buffer or workspace too small";
+        case S12_ERR_CORRUPT: return "S12_ERR_CORRUPT: container header or offsets inconsistent";
+        case S12_ERR_CUDA: return "S12_ERR_CUDA: CUDA runtime call failed";
+        case S12_ERR_DEVICE: return "S12_ERR_DEVICE: current device is not compute capability 10.0";
+        default: return "S12: unknown status";
+    }
+}
+
+int s12_device_check(void) {
+    int dev = 0, major = 0, minor = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return S12_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return S12_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return S12_ERR_CUDA;
+    return (major == 10 && minor == 0) ? S12_OK : S12_ERR_DEVICE;
+}
+
+uint64_t s12_container_bytes(int64_t rows, int64_t cols, uint64_t n_esc) {
+    if (rows <= 0 || cols <= 0 || cols % kTile) return 0;
+    return geometry(static_cast<uint64_t>(rows), static_cast<uint64_t>(cols), n_esc).total;
+}
+
+size_t s12_encode_ws_bytes(int64_t rows, int64_t cols) { return encode_ws_bytes(rows, cols); }
+
+int s12_encode(const uint16_t *w, int64_t rows, int64_t cols, void *dst, size_t dst_cap, size_t *bytes_out,
+               void *ws, size_t ws_bytes, void *stream) {
+    if (!w || !bytes_out || !ws) return S12_ERR_ARG;
+    if (rows <= 0 || cols <= 0) return S12_ERR_ARG;
+    if (cols % kTile) return S12_ERR_SHAPE;
+    if (static_cast<uint64_t>(rows) * static_cast<uint64_t>(cols) >= (uint64_t(1) << 32)) return S12_ERR_SHAPE;
+    if (!aligned16(w) || !aligned16(ws) || (dst && !aligned16(dst))) return S12_ERR_ALIGN;
+    return launch_encode(w, rows, cols, dst, dst_cap, bytes_out, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int s12_open(const void *container, size_t bytes, s12_view *out) {
+    if (!container || !out) return S12_ERR_ARG;
+    if (!aligned16(container)) return S12_ERR_ALIGN;
+    if (bytes < kHeaderBytes) return S12_ERR_CORRUPT;
+    uint8_t h[64];
+    if (cudaMemcpy(h, container, sizeof h, cudaMemcpyDeviceToHost) != cudaSuccess) return S12_ERR_CUDA;
+    if (std::memcmp(h, "S12\0", 4) != 0) return S12_ERR_CORRUPT;
+    if (get_u32(h + 4) != 1 || get_u32(h + 24) != static_cast<uint32_t>(kTile) || get_u32(h + 28) != 0)
+        return S12_ERR_CORRUPT;
+    for (int i = 40; i < 64; ++i)
+        if (h[i]) return S12_ERR_CORRUPT;
+    const uint64_t rows = get_u64(h + 8), cols = get_u64(h + 16), n_esc = get_u64(h + 32);
+    if (rows == 0 || cols == 0 || cols % kTile) return S12_ERR_CORRUPT;
+    if (rows >= (uint64_t(1) << 32) || cols >= (uint64_t(1) << 32) || rows * cols >= (uint64_t(1) << 32))
+        return S12_ERR_CORRUPT;
+    if (n_esc > rows * cols) return S12_ERR_CORRUPT;
+    const Geometry g = geometry(rows, cols, n_esc);
+    if (g.total > bytes) return S12_ERR_CORRUPT;
+    const uint8_t *c = static_cast<const uint8_t *>(container);
+    out->rows = rows;
+    out->cols = cols;
+    out->n_tiles = g.n_tiles;
+    out->n_esc = n_esc;
+    out->container_bytes = g.total;
+    out->container = container;
+    out->raw = c + g.off_raw;
+    out->code = c + g.off_code;
+    out->base = c + g.off_base;
+    out->esc_off = reinterpret_cast<const uint32_t *>(c + g.off_esc_off);
+    out->esc = reinterpret_cast<const uint16_t *>(c + g.off_esc);
+    return S12_OK;
+}
+
+int s12_decode(const s12_view *v, uint16_t *out, uint32_t *err_flag, void *stream) {
+    int rc = check_view(v);
+    if (rc != S12_OK) return rc;
+    if (!out) return S12_ERR_ARG;
+    if (!aligned16(out) || (err_flag && !aligned4(err_flag))) return S12_ERR_ALIGN;
+    return launch_decode(v, out, err_flag, static_cast<cudaStream_t>(stream));
+}
+
+int s12_gemv(const s12_view *v, const uint16_t *x, int B, float *y, uint32_t *err_flag, void *stream) {
+    int rc = check_view(v);
+    if (rc != S12_OK) return rc;
+    if (!x || !y) return S12_ERR_ARG;
+    if (B < 1 || B > S12_GEMV_MAX_BATCH) return S12_ERR_SHAPE;
+    if (v->rows > 0x7FFFFFFFull || v->cols > 0x7FFFFFFFull) return S12_ERR_SHAPE;
+    if (!aligned16(x) || !aligned4(y) || (err_flag && !aligned4(err_flag))) return S12_ERR_ALIGN;
+    return launch_gemv(v, x, B, y, err_flag, static_cast<cudaStream_t>(stream));
+}
+
+size_t s12_gemm_ws_bytes(const s12_view *v, int M) {
+    if (check_view(v) != S12_OK || M < S12_GEMM_MIN_M || M > S12_GEMM_MAX_M) return 0;
+    return gemm_ws_bytes(v, M);
+}
+
+int s12_gemm_skinny(const s12_view *v, const uint16_t *x, int M, float *y, void *ws, size_t ws_bytes,
+                    uint32_t *err_flag, void *stream) {
+    int rc = check_view(v);
+    if (rc != S12_OK) return rc;
+    if (!x || !y) return S12_ERR_ARG;
+    if (M < S12_GEMM_MIN_M || M > S12_GEMM_MAX_M) return S12_ERR_SHAPE;
+    if (v->rows > 0x7FFFFFFFull || v->cols > 0x7FFFFFFFull) return S12_ERR_SHAPE;
+    if (!aligned16(x) || !aligned4(y) || (ws && !aligned16(ws)) || (err_flag && !aligned4(err_flag)))
+        return S12_ERR_ALIGN;
+    if (ws_bytes < gemm_ws_bytes(v, M)) return S12_ERR_CAPACITY;
+    return launch_gemm(v, x, M, y, ws, ws_bytes, err_flag, static_cast<cudaStream_t>(stream));
+}
+
+size_t s12_stats_ws_bytes(void) { return 256 * sizeof(unsigned long long); }
+
+int s12_stats(const s12_view *v, s12_stats_t *out, void *ws, size_t ws_bytes, void *stream) {
+    int rc = check_view(v);
+    if (rc != S12_OK) return rc;
+    if (!out || !ws) return S12_ERR_ARG;
+    if (!aligned16(ws)) return S12_ERR_ALIGN;
+    if (ws_bytes < s12_stats_ws_bytes()) return S12_ERR_CAPACITY;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    unsigned long long *hist = static_cast<unsigned long long *>(ws);
+    rc = launch_stats_hist(v, hist, st);
+    if (rc != S12_OK) return rc;
+    unsigned long long h[256];
+    if (cudaMemcpyAsync(h, hist, sizeof h, cudaMemcpyDeviceToHost, st) != cudaSuccess) return S12_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return S12_ERR_CUDA;
+    std::memset(out, 0, sizeof *out);
+    const uint64_t nw = v->rows * v->cols;
+    out->rows = v->rows;
+    out->cols = v->cols;
+    out->n_tiles = v->n_tiles;
+    out->n_esc = v->n_esc;
+    out->container_bytes = v->container_bytes;
+    out->payload_bytes = nw + nw / 2;
+    out->header_bytes = v->n_tiles * 5;
+    out->escape_bytes = 2 * v->n_esc;
+    out->escape_rate = static_cast<double>(v->n_esc) / static_cast<double>(nw);
+    out->bits_per_weight = 8.0 * static_cast<double>(v->container_bytes) / static_cast<double>(nw);
+    out->ratio_vs_bf16 = static_cast<double>(v->container_bytes) / (2.0 * static_cast<double>(nw));
+    out->payload_ratio = static_cast<double>(out->payload_bytes) / (2.0 * static_cast<double>(nw));
+    double ent = 0.0;
+    for (int e = 0; e < 256; ++e) {
+        out->exp_hist[e] = h[e];
+        if (h[e]) {
+            const double p = static_cast<double>(h[e]) / static_cast<double>(nw);
+            ent -= p * std::log2(p);
+        }
+    }
+    out->exp_entropy_bits = ent;
+    return S12_OK;
+}
+
+int s12_bf16_gemv(const uint16_t *w, int64_t rows, int64_t cols, const uint16_t *x, int B, float *y,
+                  void *stream) {
+    if (!w || !x || !y) return S12_ERR_ARG;
+    if (rows <= 0 || cols <= 0) return S12_ERR_ARG;
+    if (cols % 8 || B < 1 || B > S12_GEMV_MAX_BATCH) return S12_ERR_SHAPE;
+    if (!aligned16(w) || !aligned16(x) || !aligned4(y)) return S12_ERR_ALIGN;
+    return launch_bf16_gemv(w, rows, cols, x, B, y, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

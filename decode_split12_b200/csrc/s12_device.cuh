@@ -1,0 +1,235 @@
+// s12_device.cuh -- device-side building blocks shared by the Split12 kernels
+// (sm_100a only): container geometry, PTX wrappers for mbarriers and TMA bulk
+// copies, bounded waits, and the register-level decode of 16 weights.
+//
+// Format (restated from the pages; see include/s12.h for the byte layout):
+// a BF16 weight is 1 sign, 8 exponent and 7 mantissa bits ("你的 bf16 模型,
+// 有 5 個 bit 是廢的", section 1 table).  It is stored as a raw byte
+// (sign | mantissa) plus a 4-bit exponent code relative to the base of its
+// 128-weight tile; code 15 means the whole value sits in the escape stream
+// ("GPU 友善 12 位無損 BF16 壓縮格式", key points and technical deep dive:
+// one integer ADD decodes, escapes live in a separate buffer).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "s12.h"
+
+namespace s12 {
+
+constexpr int kTile = 128;           // weights per tile (along K)
+constexpr int kMaxBase = 241;        // base + 14 <= 255
+constexpr uint32_t kAlign = 256;     // plane alignment inside a container
+constexpr uint32_t kHeaderBytes = 256;
+
+__host__ __device__ inline uint64_t align_up(uint64_t n, uint64_t a) { return (n + a - 1) / a * a; }
+
+// Plane offsets of a container with the given shape and escape count.
+struct Geometry {
+    uint64_t rows, cols, n_tiles, n_esc;
+    uint64_t off_raw, off_code, off_base, off_esc_off, off_esc, total;
+};
+
+__host__ __device__ inline Geometry geometry(uint64_t rows, uint64_t cols, uint64_t n_esc) {
+    Geometry g;
+    g.rows = rows;
+    g.cols = cols;
+    g.n_tiles = rows * (cols / kTile);
+    g.n_esc = n_esc;
+    g.off_raw = kHeaderBytes;
+    g.off_code = g.off_raw + align_up(rows * cols, kAlign);
+    g.off_base = g.off_code + align_up(rows * cols / 2, kAlign);
+    g.off_esc_off = g.off_base + align_up(g.n_tiles, kAlign);
+    g.off_esc = g.off_esc_off + align_up(4 * (g.n_tiles + 1), kAlign);
+    g.total = g.off_esc + align_up(2 * n_esc, kAlign);
+    return g;
+}
+
+// ---------------------------------------------------------------------------
+// Bounded waiting.  Every spin in these kernels gives up after about a second
+// at full clock, sets S12_FLAG_TIMEOUT and lets the caller unwind.
+constexpr long long kWaitCycles = 2000000000LL;
+
+__device__ __forceinline__ void raise_flag(uint32_t *err, uint32_t bits) {
+    if (err) atomicOr(err, bits);
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase with the given parity to complete.  Returns false (and
+// raises S12_FLAG_TIMEOUT) if it does not within kWaitCycles.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t *err) {
+    const uint32_t a = smem_addr(bar);
+    if (mbar_try_wait(a, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(a, parity)) {
+        if (clock64() - t0 > kWaitCycles) {
+            raise_flag(err, S12_FLAG_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+// L2 policy for data read exactly once (weights): evict first.
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ uint64_t policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// TMA bulk copy global -> shared (this CTA), completing on `bar`.
+// dst, src and bytes must be multiples of 16.
+__device__ __forceinline__ void tma_load_1d(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
+                                            uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], "
+        "%4;" ::"r"(smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Byte permute and register-level decode.
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// Four weights: raw bytes R = [r0 r1 r2 r3] and exponents E = [e0 e1 e2 e3]
+// (one per byte) give the BF16 pairs (w0, w1) and (w2, w3).  The BF16 high
+// byte is sign | exponent >> 1, the low byte is (exponent & 1) << 7 | mantissa.
+__device__ __forceinline__ void assemble4(uint32_t R, uint32_t E, uint32_t &p01, uint32_t &p23) {
+    const uint32_t M = 0x80808080u;
+    const uint32_t hi = ((E >> 1) & ~M) | (R & M);
+    const uint32_t lo = ((E << 7) & M) | (R & ~M);
+    p01 = prmt(lo, hi, 0x5140u);  // [lo0 hi0 lo1 hi1]
+    p23 = prmt(lo, hi, 0x7362u);  // [lo2 hi2 lo3 hi3]
+}
+
+// Eight weights from two raw words and one code word (byte j of C holds the
+// codes of weights 2j (low nibble) and 2j+1 (high nibble)); B4 = base in
+// every byte.  Exponent = base + code, one byte-wise integer ADD: no carry
+// leaves a byte because base <= 241 and code <= 14 on this path (escape
+// nibbles are cleared before this call whenever the word has any).
+__device__ __forceinline__ void decode8(uint32_t R0, uint32_t R1, uint32_t C, uint32_t B4, uint32_t out[4]) {
+    const uint32_t ce = (C & 0x0F0F0F0Fu) + B4;         // e0 e2 e4 e6
+    const uint32_t co = ((C >> 4) & 0x0F0F0F0Fu) + B4;  // e1 e3 e5 e7
+    const uint32_t E0 = prmt(ce, co, 0x5140u);          // e0 e1 e2 e3
+    const uint32_t E1 = prmt(ce, co, 0x7362u);          // e4 e5 e6 e7
+    assemble4(R0, E0, out[0], out[1]);
+    assemble4(R1, E1, out[2], out[3]);
+}
+
+// Sixteen weights: raw = 16 raw bytes, code = 8 code bytes; out[j] holds the
+// BF16 pair (w_2j, w_2j+1), low half first.
+__device__ __forceinline__ void decode16(uint4 raw, uint2 code, uint32_t B4, uint32_t out[8]) {
+    decode8(raw.x, raw.y, code.x, B4, out);
+    decode8(raw.z, raw.w, code.y, B4, out + 4);
+}
+
+// Bit 4j+3 set iff nibble j of C equals 15 (an escape).
+__device__ __forceinline__ uint32_t escape_nibbles(uint32_t C) {
+    return ((C & 0x77777777u) + 0x11111111u) & C & 0x88888888u;
+}
+
+// Clear every escape nibble (so the byte-wise ADD cannot carry).
+__device__ __forceinline__ uint32_t clear_escapes(uint32_t C, uint32_t m) {
+    return C & ~(m | (m >> 1) | (m >> 2) | (m >> 3));
+}
+
+// Replace the weights flagged in (m0, m1) by consecutive escape-stream
+// values starting at index `first`; `limit` is one past the last index this
+// tile may read (tile end, clamped to the stream).  Out-of-range reads are
+// skipped and flagged.
+__device__ __forceinline__ void patch_escapes(uint32_t out[8], uint32_t m0, uint32_t m1, uint64_t first,
+                                              uint64_t limit, const uint16_t *__restrict__ esc, uint32_t *err) {
+    uint64_t idx = first;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        const uint32_t m = (j < 8) ? m0 : m1;
+        if (m & (8u << (4 * (j & 7)))) {
+            uint32_t v = 0;
+            if (idx < limit) {
+                v = __ldg(esc + idx);
+            } else {
+                raise_flag(err, S12_FLAG_ESC_RANGE);
+            }
+            ++idx;
+            if (j & 1)
+                out[j >> 1] = (out[j >> 1] & 0x0000FFFFu) | (v << 16);
+            else
+                out[j >> 1] = (out[j >> 1] & 0xFFFF0000u) | v;
+        }
+    }
+}
+
+// Warp-collective escape fix-up for one 16-weight chunk per lane.  The warp
+// covers up to four tiles, eight lanes per tile.  `lo`/`hi` are esc_off[t]
+// and esc_off[t+1] of the lane's tile (read by every lane).  Must be called
+// by all 32 lanes (inactive lanes pass m0 = m1 = 0).  Re-decodes the chunk
+// with escape nibbles cleared and patches the escaped weights; checks each
+// tile's code-15 count against its offsets.
+__device__ __forceinline__ void fix_escapes(uint32_t out[8], uint4 raw, uint2 code, uint32_t B4, uint32_t m0,
+                                            uint32_t m1, uint32_t lo, uint32_t hi, bool active, uint64_t n_esc,
+                                            const uint16_t *__restrict__ esc, uint32_t *err) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t cnt = __popc(m0) + __popc(m1);
+    uint32_t incl = cnt;
+#pragma unroll
+    for (int d = 1; d < 8; d <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, d, 8);
+        if ((lane & 7) >= d) incl += v;
+    }
+    const uint32_t total = __shfl_sync(0xFFFFFFFFu, incl, 7, 8);
+    if (!active) return;
+    if ((lane & 7) == 0 && hi - lo != total) raise_flag(err, S12_FLAG_ESC_COUNT);
+    if (cnt == 0) return;
+    uint2 c2 = make_uint2(clear_escapes(code.x, m0), clear_escapes(code.y, m1));
+    decode16(raw, c2, B4, out);
+    uint64_t limit = hi < n_esc ? hi : n_esc;
+    if (lo > hi) limit = 0;
+    patch_escapes(out, m0, m1, static_cast<uint64_t>(lo) + (incl - cnt), limit, esc, err);
+}
+
+}  // namespace s12

@@ -1,0 +1,25 @@
+// s12_launch.h -- internal host-side declarations of the kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "s12.h"
+
+namespace s12 {
+
+// Number of SMs of the current device (cached per device).
+cudaError_t device_sms(int *sms);
+
+int launch_decode(const s12_view *v, uint16_t *out, uint32_t *err, cudaStream_t stream);
+int launch_gemv(const s12_view *v, const uint16_t *x, int B, float *y, uint32_t *err, cudaStream_t stream);
+int launch_bf16_gemv(const uint16_t *w, int64_t rows, int64_t cols, const uint16_t *x, int B, float *y,
+                     cudaStream_t stream);
+size_t encode_ws_bytes(int64_t rows, int64_t cols);
+int launch_encode(const uint16_t *w, int64_t rows, int64_t cols, void *dst, size_t dst_cap, size_t *bytes_out,
+                  void *ws, size_t ws_bytes, cudaStream_t stream);
+int launch_stats_hist(const s12_view *v, unsigned long long *hist_dev, cudaStream_t stream);
+size_t gemm_ws_bytes(const s12_view *v, int M);
+int launch_gemm(const s12_view *v, const uint16_t *x, int M, float *y, void *ws, size_t ws_bytes, uint32_t *err,
+                cudaStream_t stream);
+
+}  // namespace s12

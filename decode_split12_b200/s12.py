@@ -1,0 +1,255 @@
+"""Thin ctypes binding of libs12.so (C ABI in include/s12.h).
+
+Argument marshalling only: every step of the compute path runs in the CUDA
+library.  torch provides device memory and streams.  The functions keep the
+C names (``s12_encode``, ``s12_open``, ``s12_decode``, ``s12_gemv``,
+``s12_gemm_skinny``, ``s12_stats``, ``s12_bf16_gemv``).
+
+There is no CPU fallback: if libs12.so is missing or the device is not a
+B200-class part, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libs12.so")
+
+S12_OK = 0
+S12_ERR_ARG = 1
+S12_ERR_SHAPE = 2
+S12_ERR_ALIGN = 3
+S12_ERR_CAPACITY = 4
+S12_ERR_CORRUPT = 5
+S12_ERR_CUDA = 6
+S12_ERR_DEVICE = 7
+
+S12_FLAG_ESC_COUNT = 1
+S12_FLAG_ESC_RANGE = 2
+S12_FLAG_BASE = 4
+S12_FLAG_TIMEOUT = 8
+
+EXPORTED = (
+    "s12_error_string", "s12_device_check", "s12_container_bytes", "s12_encode_ws_bytes", "s12_encode",
+    "s12_open", "s12_decode", "s12_gemv", "s12_gemm_ws_bytes", "s12_gemm_skinny", "s12_stats_ws_bytes",
+    "s12_stats", "s12_bf16_gemv",
+)
+
+
+class S12Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        msg = _lib().s12_error_string(status).decode() if _LIB is not None else str(status)
+        super().__init__(f"{what}: {msg}")
+        self.status = status
+
+
+class View(C.Structure):
+    _fields_ = [
+        ("rows", C.c_uint64), ("cols", C.c_uint64), ("n_tiles", C.c_uint64), ("n_esc", C.c_uint64),
+        ("container_bytes", C.c_uint64), ("container", C.c_void_p), ("raw", C.c_void_p),
+        ("code", C.c_void_p), ("base", C.c_void_p), ("esc_off", C.c_void_p), ("esc", C.c_void_p),
+    ]
+
+
+class Stats(C.Structure):
+    _fields_ = [
+        ("rows", C.c_uint64), ("cols", C.c_uint64), ("n_tiles", C.c_uint64), ("n_esc", C.c_uint64),
+        ("container_bytes", C.c_uint64), ("payload_bytes", C.c_uint64), ("header_bytes", C.c_uint64),
+        ("escape_bytes", C.c_uint64), ("escape_rate", C.c_double), ("bits_per_weight", C.c_double),
+        ("ratio_vs_bf16", C.c_double), ("payload_ratio", C.c_double), ("exp_entropy_bits", C.c_double),
+        ("exp_hist", C.c_uint64 * 256),
+    ]
+
+
+_LIB = None
+_P = C.c_void_p
+_I64 = C.c_int64
+_SZ = C.c_size_t
+
+
+def _lib() -> C.CDLL:
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libs12.so not built ({LIB_PATH}); run __graft_entry__.build()")
+        lib = C.CDLL(LIB_PATH)
+        lib.s12_error_string.argtypes = [C.c_int]
+        lib.s12_error_string.restype = C.c_char_p
+        lib.s12_device_check.argtypes = []
+        lib.s12_device_check.restype = C.c_int
+        lib.s12_container_bytes.argtypes = [_I64, _I64, C.c_uint64]
+        lib.s12_container_bytes.restype = C.c_uint64
+        lib.s12_encode_ws_bytes.argtypes = [_I64, _I64]
+        lib.s12_encode_ws_bytes.restype = _SZ
+        lib.s12_encode.argtypes = [_P, _I64, _I64, _P, _SZ, C.POINTER(_SZ), _P, _SZ, _P]
+        lib.s12_encode.restype = C.c_int
+        lib.s12_open.argtypes = [_P, _SZ, C.POINTER(View)]
+        lib.s12_open.restype = C.c_int
+        lib.s12_decode.argtypes = [C.POINTER(View), _P, _P, _P]
+        lib.s12_decode.restype = C.c_int
+        lib.s12_gemv.argtypes = [C.POINTER(View), _P, C.c_int, _P, _P, _P]
+        lib.s12_gemv.restype = C.c_int
+        lib.s12_gemm_ws_bytes.argtypes = [C.POINTER(View), C.c_int]
+        lib.s12_gemm_ws_bytes.restype = _SZ
+        lib.s12_gemm_skinny.argtypes = [C.POINTER(View), _P, C.c_int, _P, _P, _SZ, _P, _P]
+        lib.s12_gemm_skinny.restype = C.c_int
+        lib.s12_stats_ws_bytes.argtypes = []
+        lib.s12_stats_ws_bytes.restype = _SZ
+        lib.s12_stats.argtypes = [C.POINTER(View), C.POINTER(Stats), _P, _SZ, _P]
+        lib.s12_stats.restype = C.c_int
+        lib.s12_bf16_gemv.argtypes = [_P, _I64, _I64, _P, C.c_int, _P, _P]
+        lib.s12_bf16_gemv.restype = C.c_int
+        _LIB = lib
+    return _LIB
+
+
+def lib() -> C.CDLL:
+    return _lib()
+
+
+def _check(rc: int, what: str):
+    if rc != S12_OK:
+        raise S12Error(rc, what)
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream)
+
+
+def _dptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return C.c_void_p(t.data_ptr())
+
+
+def _u16(t: torch.Tensor) -> torch.Tensor:
+    """BF16 / int16 / uint16 tensors viewed as their 16-bit patterns."""
+    if t.dtype in (torch.bfloat16, torch.int16, torch.float16):
+        return t
+    if t.dtype == torch.uint16:
+        return t
+    raise TypeError(f"expected a 16-bit tensor, got {t.dtype}")
+
+
+class Container:
+    """A Split12 container in device memory plus its opened view."""
+
+    def __init__(self, blob: torch.Tensor):
+        self.blob = blob
+        self.view = s12_open(blob)
+
+    @property
+    def rows(self):
+        return int(self.view.rows)
+
+    @property
+    def cols(self):
+        return int(self.view.cols)
+
+    @property
+    def n_esc(self):
+        return int(self.view.n_esc)
+
+    @property
+    def nbytes(self):
+        return int(self.view.container_bytes)
+
+
+def device_check():
+    _check(_lib().s12_device_check(), "s12_device_check")
+
+
+def s12_container_bytes(rows: int, cols: int, n_esc: int) -> int:
+    return int(_lib().s12_container_bytes(rows, cols, n_esc))
+
+
+def s12_encode(w: torch.Tensor, ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Encode a (rows, cols) BF16 CUDA tensor; returns the container as a
+    uint8 CUDA tensor (two library calls: size query, then encode)."""
+    w = _u16(w)
+    rows, cols = w.shape
+    lib_ = _lib()
+    need_ws = lib_.s12_encode_ws_bytes(rows, cols)
+    if ws is None:
+        ws = torch.empty(max(need_ws, 256), dtype=torch.uint8, device=w.device)
+    st = _stream(stream)
+    nbytes = _SZ(0)
+    _check(lib_.s12_encode(_dptr(w), rows, cols, None, 0, C.byref(nbytes), _dptr(ws), ws.numel(), st),
+           "s12_encode(size)")
+    blob = torch.empty(nbytes.value, dtype=torch.uint8, device=w.device)
+    _check(lib_.s12_encode(_dptr(w), rows, cols, _dptr(blob), blob.numel(), C.byref(nbytes), _dptr(ws),
+                           ws.numel(), st), "s12_encode")
+    return blob
+
+
+def s12_open(blob: torch.Tensor) -> View:
+    v = View()
+    _check(_lib().s12_open(_dptr(blob), blob.numel() * blob.element_size(), C.byref(v)), "s12_open")
+    return v
+
+
+def s12_decode(view: View, out: torch.Tensor | None = None, err_flag: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty((view.rows, view.cols), dtype=torch.bfloat16, device="cuda")
+    _check(_lib().s12_decode(C.byref(view), _dptr(out), _dptr(err_flag), _stream(stream)), "s12_decode")
+    return out
+
+
+def s12_gemv(view: View, x: torch.Tensor, y: torch.Tensor | None = None, err_flag: torch.Tensor | None = None,
+             stream=None) -> torch.Tensor:
+    x = _u16(x)
+    B = x.shape[0] if x.dim() == 2 else 1
+    if y is None:
+        y = torch.empty((B, view.rows), dtype=torch.float32, device=x.device)
+    _check(_lib().s12_gemv(C.byref(view), _dptr(x), B, _dptr(y), _dptr(err_flag), _stream(stream)), "s12_gemv")
+    return y
+
+
+def s12_gemm_ws_bytes(view: View, M: int) -> int:
+    return int(_lib().s12_gemm_ws_bytes(C.byref(view), M))
+
+
+def s12_gemm_skinny(view: View, x: torch.Tensor, y: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                    err_flag: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    x = _u16(x)
+    M = x.shape[0]
+    if y is None:
+        y = torch.empty((M, view.rows), dtype=torch.float32, device=x.device)
+    need = s12_gemm_ws_bytes(view, M)
+    if ws is None:
+        ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=x.device)
+    _check(_lib().s12_gemm_skinny(C.byref(view), _dptr(x), M, _dptr(y), _dptr(ws), ws.numel(), _dptr(err_flag),
+                                  _stream(stream)), "s12_gemm_skinny")
+    return y
+
+
+def s12_stats(view: View, ws: torch.Tensor | None = None, stream=None) -> dict:
+    lib_ = _lib()
+    if ws is None:
+        ws = torch.empty(lib_.s12_stats_ws_bytes(), dtype=torch.uint8, device="cuda")
+    st = Stats()
+    _check(lib_.s12_stats(C.byref(view), C.byref(st), _dptr(ws), ws.numel(), _stream(stream)), "s12_stats")
+    d = {name: getattr(st, name) for name, _ in Stats._fields_ if name != "exp_hist"}
+    d["exp_hist"] = list(st.exp_hist[:])
+    return d
+
+
+def s12_bf16_gemv(w: torch.Tensor, x: torch.Tensor, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    w = _u16(w)
+    x = _u16(x)
+    rows, cols = w.shape
+    B = x.shape[0] if x.dim() == 2 else 1
+    if y is None:
+        y = torch.empty((B, rows), dtype=torch.float32, device=x.device)
+    _check(_lib().s12_bf16_gemv(_dptr(w), rows, cols, _dptr(x), B, _dptr(y), _stream(stream)), "s12_bf16_gemv")
+    return y

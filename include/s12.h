@@ -1,0 +1,209 @@
+/*
+ * s12.h -- C ABI of the Split12 library (libs12.so): lossless 12-bit BF16
+ * weights decoded on the GPU and fused into the matrix-vector and skinny
+ * matrix products of LLM decoding.  Built for NVIDIA B200 (sm_100a) only.
+ *
+ * Sources (web pages, cited by title and section):
+ *   [W] "Lossless LLM Weight Compression vs 8-bit GGUF: What Is Ready for
+ *       Production?" (wavect.io blog, with its Chinese and German editions).
+ *   [M] "你的 bf16 模型,有 5 個 bit 是廢的" (meowlab blog, 2026-10-04).
+ *   [T] "GPU 友善 12 位無損 BF16 壓縮格式" (setupai.cc digest of a Reddit post
+ *       on a GPU-friendly 12-bit lossless BF16 format).
+ *
+ * FORMAT ("Split12 container").  A BF16 weight has 1 sign, 8 exponent and 7
+ * mantissa bits ([M] section 1 table).  Trained weights use few exponents,
+ * so common exponents get short fixed codes and rare ones go to an exact
+ * escape stream ([W] "What did the GLM-5.2 experiment actually prove?").
+ * Here each weight w becomes
+ *     raw  = ((w >> 8) & 0x80) | (w & 0x7F)      one byte: sign + mantissa
+ *     code = e - base  (0..14)  or 15 (escape)   one nibble, e = (w>>7)&0xFF
+ * for a base shared by a tile of 128 weights along a row ([T] technical deep
+ * dive: blocks of 128 weights share a base), chosen as the smallest base in
+ * [0, 241] whose window [base, base+14] holds the most of the tile's
+ * exponents.  Decoding is one integer ADD, exponent = base + code ([T] key
+ * points).  Escaped weights are stored whole in a separate stream ([T]
+ * technical deep dive), in row-major order, located through per-tile prefix
+ * offsets.  That is 12 bits per weight plus 5 header bytes per tile and 2
+ * bytes per escape ([T] key points: fixed 12-bit rate, 1.33x smaller).
+ *
+ * Container bytes (little-endian; every part starts at a multiple of 256
+ * bytes from the start and is zero-padded to a multiple of 256 bytes):
+ *     header  64 bytes used: "S12\0", u32 version=1, u64 rows, u64 cols,
+ *             u32 tile=128, u32 flags=0, u64 n_esc, zeros
+ *     raw     u8 [rows*cols]          row-major
+ *     code    u8 [rows*cols/2]        even weight in the low nibble
+ *     base    u8 [n_tiles]            tile t = r*(cols/128) + j covers
+ *                                     w[r][128j .. 128j+127]
+ *     esc_off u32[n_tiles+1]          escapes before tile t; last = n_esc
+ *     esc     u16[n_esc]              escaped BF16 values
+ *
+ * CONVENTIONS
+ *   - Every call returns an s12 status (0 = S12_OK).
+ *   - Pointers marked "device" are CUDA device pointers on the current
+ *     device; the caller allocates and owns all of them.  The library never
+ *     allocates or frees device memory.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Kernel calls are enqueued on it and return at once, except
+ *     where a call says it synchronises.
+ *   - Device pointers must be 16-byte aligned unless stated otherwise.
+ *   - `err_flag` (device, u32, nullable): kernels that read a container
+ *     OR into it S12_FLAG_* bits when they meet corrupt data.  They never
+ *     trap or hang: the offending escape index is clamped and work goes on.
+ *     The caller reads the word back (and clears it) when it wants to.
+ *   - The library keeps no mutable global state and is thread-safe.
+ */
+#ifndef S12_H
+#define S12_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ---- */
+#define S12_OK 0
+#define S12_ERR_ARG 1      /* null pointer or negative / zero size           */
+#define S12_ERR_SHAPE 2    /* cols % 128 != 0, batch out of range, too large */
+#define S12_ERR_ALIGN 3    /* a device pointer is not 16-byte aligned        */
+#define S12_ERR_CAPACITY 4 /* destination or workspace too small             */
+#define S12_ERR_CORRUPT 5  /* container header or offsets inconsistent       */
+#define S12_ERR_CUDA 6     /* a CUDA runtime call failed                     */
+#define S12_ERR_DEVICE 7   /* current device is not compute capability 10.0  */
+
+/* ---- err_flag bits set by kernels ---- */
+#define S12_FLAG_ESC_COUNT 1u   /* a tile's code-15 count != its esc_off span */
+#define S12_FLAG_ESC_RANGE 2u   /* esc_off points outside the escape stream   */
+#define S12_FLAG_BASE 4u        /* a tile base above 241                      */
+#define S12_FLAG_TIMEOUT 8u     /* a bounded wait inside a kernel gave up     */
+
+#define S12_TILE 128
+#define S12_GEMV_MAX_BATCH 8
+#define S12_GEMM_MIN_M 16
+#define S12_GEMM_MAX_M 256
+
+/* Host-side description of an opened container.  All pointers are device
+ * pointers into the caller's container buffer. */
+typedef struct s12_view {
+    uint64_t rows;            /* output features (N)                      */
+    uint64_t cols;            /* input features (K), multiple of 128      */
+    uint64_t n_tiles;         /* rows * cols / 128                        */
+    uint64_t n_esc;           /* escaped weights                          */
+    uint64_t container_bytes; /* total size, multiple of 256              */
+    const void *container;    /* start of the container                   */
+    const uint8_t *raw;       /* u8 [rows*cols]                           */
+    const uint8_t *code;      /* u8 [rows*cols/2]                         */
+    const uint8_t *base;      /* u8 [n_tiles]                             */
+    const uint32_t *esc_off;  /* u32[n_tiles+1]                           */
+    const uint16_t *esc;      /* u16[n_esc]                               */
+} s12_view;
+
+typedef struct s12_stats_t {
+    uint64_t rows, cols, n_tiles, n_esc;
+    uint64_t container_bytes; /* everything, padding included            */
+    uint64_t payload_bytes;   /* raw + code = 1.5 bytes per weight       */
+    uint64_t header_bytes;    /* 5 bytes per tile (base + offset)        */
+    uint64_t escape_bytes;    /* 2 bytes per escape                      */
+    double escape_rate;       /* n_esc / (rows*cols)                     */
+    double bits_per_weight;   /* 8 * container_bytes / (rows*cols)       */
+    double ratio_vs_bf16;     /* container_bytes / (2*rows*cols)         */
+    double payload_ratio;     /* payload_bytes / (2*rows*cols) = 0.75    */
+    double exp_entropy_bits;  /* Shannon entropy of the exponent field   */
+    uint64_t exp_hist[256];   /* histogram of decoded exponent fields    */
+} s12_stats_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *s12_error_string(int status);
+
+/* S12_OK when the current device is a B200-class part (compute capability
+ * 10.0, sm_100a code in this library), S12_ERR_DEVICE otherwise. */
+int s12_device_check(void);
+
+/* Container size in bytes for a shape and escape count (closed form of the
+ * layout above); 0 when the shape is invalid (cols % 128 != 0 or zero). */
+uint64_t s12_container_bytes(int64_t rows, int64_t cols, uint64_t n_esc);
+
+/* ---- encoder ([W] "What did the GLM-5.2 experiment actually prove?":
+ * short codes for common exponents, rare ones to an exact escape stream;
+ * [T] technical deep dive: 128-weight blocks with a shared base) ---- */
+
+/* Workspace bytes s12_encode needs for this shape (device scratch, any
+ * content, 16-byte aligned, owned by the caller). */
+size_t s12_encode_ws_bytes(int64_t rows, int64_t cols);
+
+/* Encode a row-major BF16 matrix `w` (device, rows x cols, cols % 128 == 0,
+ * rows*cols < 2^32) into a Split12 container.
+ *   dst == NULL: only computes *bytes_out (the exact container size).
+ *   dst != NULL: writes the whole container (header, planes, zero padding)
+ *                to dst (device, dst_cap bytes); S12_ERR_CAPACITY when
+ *                dst_cap < the size.
+ * Both forms run the per-tile histogram/window and escape-count kernels and
+ * then SYNCHRONISE `stream` once to read the escape total; the packing
+ * kernels of the second form are then enqueued asynchronously.
+ * The result is byte-for-byte the same container on every call. */
+int s12_encode(const uint16_t *w, int64_t rows, int64_t cols, void *dst, size_t dst_cap,
+               size_t *bytes_out, void *ws, size_t ws_bytes, void *stream);
+
+/* Validate the 64-byte header of a container (device, `bytes` long) and
+ * fill *out with its shape and plane pointers.  Copies the header to the
+ * host and so SYNCHRONISES (the legacy default stream).  S12_ERR_CORRUPT on
+ * a bad magic, version, tile size, flags, shape or a size above `bytes`. */
+int s12_open(const void *container, size_t bytes, s12_view *out);
+
+/* ---- standalone decode ([T] key points: one integer ADD per weight,
+ * code 15 read from the escape stream) ---- */
+
+/* Decode the whole container to BF16 `out` (device, rows x cols, row-major).
+ * Bit-exact: out equals the encoded matrix. */
+int s12_decode(const s12_view *v, uint16_t *out, uint32_t *err_flag, void *stream);
+
+/* ---- fused decode-GEMV ([W] "What does 'lossless' mean for LLM weights?":
+ * decode the exact BF16 values into registers or shared memory and use them
+ * at once in the matrix product) ---- */
+
+/* y[b][n] = sum_k W[n][k] * x[b][k] for b < B, 1 <= B <= 8.
+ *   x: device BF16, B x cols row-major.   y: device FP32, B x rows
+ *   row-major (4-byte alignment suffices), overwritten.
+ * Weights are decoded in registers from shared-memory tiles staged by the
+ * TMA engine and multiplied in FP32; the sum order is fixed, so repeated
+ * calls give identical y. */
+int s12_gemv(const s12_view *v, const uint16_t *x, int B, float *y, uint32_t *err_flag,
+             void *stream);
+
+/* ---- fused decode-skinny-GEMM on tcgen05 tensor cores ---- */
+
+/* Workspace bytes s12_gemm_skinny needs for this container and M. */
+size_t s12_gemm_ws_bytes(const s12_view *v, int M);
+
+/* y[m][n] = sum_k W[n][k] * x[m][k] for 16 <= M <= 256.
+ *   x: device BF16, M x cols row-major.  y: device FP32, M x rows row-major,
+ *   overwritten.  ws: device scratch of s12_gemm_ws_bytes(v, M) bytes.
+ * Decoded BF16 tiles are written to shared memory and multiplied by the
+ * tensor cores with FP32 accumulation. */
+int s12_gemm_skinny(const s12_view *v, const uint16_t *x, int M, float *y, void *ws,
+                    size_t ws_bytes, uint32_t *err_flag, void *stream);
+
+/* ---- statistics ([M] section 1: exponent entropy; [T] key points:
+ * escape rate) ---- */
+
+/* Workspace bytes s12_stats needs (device scratch). */
+size_t s12_stats_ws_bytes(void);
+
+/* Fill *out with sizes, rates and the exponent histogram/entropy of the
+ * decoded weights.  Runs a histogram kernel and SYNCHRONISES `stream`. */
+int s12_stats(const s12_view *v, s12_stats_t *out, void *ws, size_t ws_bytes, void *stream);
+
+/* ---- uncompressed baseline ---- */
+
+/* Plain BF16 GEMV, the comparison point for s12_gemv: y[b][n] =
+ * sum_k w[n][k] * x[b][k], w device BF16 rows x cols (cols % 8 == 0),
+ * 1 <= B <= 8, y FP32 B x rows. */
+int s12_bf16_gemv(const uint16_t *w, int64_t rows, int64_t cols, const uint16_t *x, int B,
+                  float *y, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* S12_H */
