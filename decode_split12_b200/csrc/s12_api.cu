@@ -3,6 +3,9 @@
 #include <atomic>
 #include <cmath>
 #include <cstring>
+#include <mutex>
+
+#include <cudaTypedefs.h>
 
 #include "s12_device.cuh"
 #include "s12_launch.h"
@@ -46,6 +49,31 @@ cudaError_t device_sms(int *sms) {
     if (dev >= 0 && dev < kMaxDevices) g_sms[dev].store(n, std::memory_order_relaxed);
     *sms = n;
     return cudaSuccess;
+}
+
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
+std::once_flag g_encode_once;
+}  // namespace
+
+int make_tmap_u64_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t rows, uint64_t row_stride,
+                     uint32_t box_inner, uint32_t box_rows) {
+    std::call_once(g_encode_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode_tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    if (!g_encode_tiled) return S12_ERR_CUDA;
+    const cuuint64_t dims[2] = {inner, rows};
+    const cuuint64_t strides[1] = {row_stride};
+    const cuuint32_t box[2] = {box_inner, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode_tiled(out, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<void *>(base), dims, strides, box,
+                                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? S12_OK : S12_ERR_CUDA;
 }
 
 }  // namespace s12

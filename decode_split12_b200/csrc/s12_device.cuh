@@ -88,19 +88,48 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait that lets the hardware suspend the thread for up to `ns`
+// nanoseconds while the phase is pending (no issue slots burnt spinning).
+__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete.  Returns false (and
 // raises S12_FLAG_TIMEOUT) if it does not within kWaitCycles.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t *err) {
     const uint32_t a = smem_addr(bar);
     if (mbar_try_wait(a, parity)) return true;
     const long long t0 = clock64();
+#ifndef S12_WAIT_MODE
+#define S12_WAIT_MODE 1
+#endif
+#if S12_WAIT_MODE == 0
+    while (!mbar_try_wait_hint(a, parity, 20000u)) {
+#else
     while (!mbar_try_wait(a, parity)) {
+#endif
         if (clock64() - t0 > kWaitCycles) {
             raise_flag(err, S12_FLAG_TIMEOUT);
             return false;
         }
     }
     return true;
+}
+
+// Programmatic dependent launch: wait until the grids this one depends on
+// have completed (and their writes are visible); allow the next grid in the
+// stream to begin launching.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // L2 policy for data read exactly once (weights): evict first.
@@ -125,6 +154,21 @@ __device__ __forceinline__ void tma_load_1d(void *dst, const void *src, uint32_t
         "%4;" ::"r"(smem_addr(dst)),
         "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
         : "memory");
+}
+
+// TMA tiled copy of a 2-D box (coordinates in elements, innermost first)
+// global -> shared (this CTA), completing on `bar`.  No multicast.
+__device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, int c0, int c1, uint64_t *bar,
+                                            uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
+        "l"(tmap), "r"(c0), "r"(c1), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const void *tmap) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -182,8 +226,12 @@ __device__ __forceinline__ uint32_t clear_escapes(uint32_t C, uint32_t m) {
 // values starting at index `first`; `limit` is one past the last index this
 // tile may read (tile end, clamped to the stream).  Out-of-range reads are
 // skipped and flagged.
+// If `staged` is set, escapes [stage_lo, stage_hi) are also in shared memory
+// at `esc_smem` (element stage_lo first) and are read from there.
 __device__ __forceinline__ void patch_escapes(uint32_t out[8], uint32_t m0, uint32_t m1, uint64_t first,
-                                              uint64_t limit, const uint16_t *__restrict__ esc, uint32_t *err) {
+                                              uint64_t limit, const uint16_t *__restrict__ esc, uint32_t *err,
+                                              const uint16_t *esc_smem = nullptr, uint64_t stage_lo = 0,
+                                              uint64_t stage_hi = 0) {
     uint64_t idx = first;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
@@ -191,7 +239,10 @@ __device__ __forceinline__ void patch_escapes(uint32_t out[8], uint32_t m0, uint
         if (m & (8u << (4 * (j & 7)))) {
             uint32_t v = 0;
             if (idx < limit) {
-                v = __ldg(esc + idx);
+                if (esc_smem && idx >= stage_lo && idx < stage_hi)
+                    v = esc_smem[idx - stage_lo];
+                else
+                    v = __ldg(esc + idx);
             } else {
                 raise_flag(err, S12_FLAG_ESC_RANGE);
             }
@@ -204,15 +255,18 @@ __device__ __forceinline__ void patch_escapes(uint32_t out[8], uint32_t m0, uint
     }
 }
 
-// Warp-collective escape fix-up for one 16-weight chunk per lane.  The warp
+// Warp-collective escape fix-up for one 16-weight chunk per lane (kept out
+// of line: it is the rare path, and inlining it bloats the hot loops).  The warp
 // covers up to four tiles, eight lanes per tile.  `lo`/`hi` are esc_off[t]
 // and esc_off[t+1] of the lane's tile (read by every lane).  Must be called
 // by all 32 lanes (inactive lanes pass m0 = m1 = 0).  Re-decodes the chunk
 // with escape nibbles cleared and patches the escaped weights; checks each
 // tile's code-15 count against its offsets.
-__device__ __forceinline__ void fix_escapes(uint32_t out[8], uint4 raw, uint2 code, uint32_t B4, uint32_t m0,
+static __device__ __noinline__ void fix_escapes(uint32_t out[8], uint4 raw, uint2 code, uint32_t B4, uint32_t m0,
                                             uint32_t m1, uint32_t lo, uint32_t hi, bool active, uint64_t n_esc,
-                                            const uint16_t *__restrict__ esc, uint32_t *err) {
+                                            const uint16_t *__restrict__ esc, uint32_t *err,
+                                            const uint16_t *esc_smem = nullptr, uint64_t stage_lo = 0,
+                                            uint64_t stage_hi = 0) {
     const int lane = threadIdx.x & 31;
     const uint32_t cnt = __popc(m0) + __popc(m1);
     uint32_t incl = cnt;
@@ -229,7 +283,8 @@ __device__ __forceinline__ void fix_escapes(uint32_t out[8], uint4 raw, uint2 co
     decode16(raw, c2, B4, out);
     uint64_t limit = hi < n_esc ? hi : n_esc;
     if (lo > hi) limit = 0;
-    patch_escapes(out, m0, m1, static_cast<uint64_t>(lo) + (incl - cnt), limit, esc, err);
+    patch_escapes(out, m0, m1, static_cast<uint64_t>(lo) + (incl - cnt), limit, esc, err, esc_smem, stage_lo,
+                  stage_hi);
 }
 
 }  // namespace s12

@@ -1,6 +1,7 @@
 // s12_launch.h -- internal host-side declarations of the kernel launchers.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "s12.h"
@@ -9,6 +10,12 @@ namespace s12 {
 
 // Number of SMs of the current device (cached per device).
 cudaError_t device_sms(int *sms);
+
+// Tiled TMA descriptor for a row-major 2-D array of 8-byte elements:
+// `inner` elements per row, `rows` rows, `row_stride` bytes between rows,
+// box of box_inner x box_rows elements, out-of-bounds elements read as 0.
+int make_tmap_u64_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t rows, uint64_t row_stride,
+                     uint32_t box_inner, uint32_t box_rows);
 
 int launch_decode(const s12_view *v, uint16_t *out, uint32_t *err, cudaStream_t stream);
 int launch_gemv(const s12_view *v, const uint16_t *x, int B, float *y, uint32_t *err, cudaStream_t stream);
