@@ -6,86 +6,90 @@
 // registers and used at once in the product ("Lossless LLM Weight
 // Compression vs 8-bit GGUF", section "What does 'lossless' mean for LLM
 // weights?": decode into registers or shared memory and multiply
-// immediately).  The kernel is HBM-bound: it must move the compressed planes
+// immediately).  The kernel is HBM-bound and must move the compressed planes
 // (1.5 bytes per weight + 5 bytes per tile + 2 bytes per escape) at close to
-// the copy bandwidth.
+// the copy bandwidth, so the work per weight has to stay at a few integer
+// instructions.
 //
-// Work: a CTA owns a contiguous range of rows (one persistent CTA per SM).
-// Each row is cut into passes of up to 4 tiles (512 columns); the CTA's
-// passes, in row-major order, are dealt to its NW warps in contiguous, equal
-// ranges, so every warp streams the same number of bytes and no warp waits
-// for another.  The activations x are staged once per CTA in shared memory
-// by the TMA engine (a bulk copy per batch row).
+// Shape of the work.  A "block" is 16 rows x one 128-weight tile column.  A
+// warp decodes a block straight into the A-operand registers of the warp-level
+// tensor-core product mma.m16n8k16 (BF16 in, FP32 accumulate).  Lane (g, q)
+// (g = lane / 4, q = lane % 4) owns rows g and g+8 and the 32 columns
+// 32q .. 32q+31 of the tile, as two 16-weight chunks (halves h = 0, 1).  A
+// chunk is decoded with a byte-wise base + code ADD and byte permutes into
+// eight BF16 pairs that feed four products; the B operand is the matching
+// slice of x for batch row g.  The tensor core does the multiplies and the
+// reduction across the quad, so the decode is nearly all the arithmetic.
 //
-// A warp streams its range U passes at a time: every lane first issues the
-// loads of its 16 weights of each of the U passes (one 128-bit load of raw
-// bytes, one 64-bit load of codes, the tile's base byte and escape offsets;
-// streaming cache policy), then decodes them -- a byte-wise base + code ADD
-// and byte permutes into BF16 pairs -- and multiplies them with the BF16
-// activations by FMAs that take BF16 inputs and accumulate in FP32, one
-// accumulator set per pass.  Many warps per SM keep enough loads in flight
-// to cover the HBM latency.  The passes' sums are then folded into rows:
-// when the row changes the warp reduces with shuffles; rows wholly inside
-// its range go straight to y, the at most two rows it shares with
-// neighbouring warps are combined at the end in warp order, so y is
-// deterministic.  Code-15 weights take their exact value from the escape
-// stream (rare, out-of-line path).
+// Data movement.  Every warp owns a ring of shared-memory stages.  One lane
+// fills a stage with two TMA tensor copies (raw plane: 16 rows x 128 bytes
+// with the 128-byte swizzle, so the lanes' 16-byte reads hit distinct banks;
+// code plane: 16 rows x 64 bytes), completing on the stage's mbarrier, and
+// refills it as soon as the lanes have read it into registers.  The ring
+// keeps several blocks in flight per warp at no register cost, so 16 warps
+// fit on an SM.  The per-tile base and escape offsets are read with plain
+// loads two blocks ahead, and the first escape value of a tile that has
+// escapes is fetched one block ahead, so escapes rarely stall a warp.
 //
-// Launched with programmatic dependent launch: the weight loads of a CTA's
-// first passes may start before the previous kernel in the stream has
-// finished; x and y wait for it.
+// Work split (stream-K).  Blocks are numbered row-group-major (16-row group,
+// then tile column) and dealt to all warps of the grid in equal contiguous
+// ranges, so every warp streams the same number of bytes.  A warp keeps the
+// accumulators of its current row group in registers; a group it covers
+// whole goes straight to y.  A group shared by several warps is finished by
+// the last of them to arrive: each contributor writes its partial to the
+// workspace and bumps the group's counter; the one that completes the count
+// adds the partials in warp order (so y is the same on every call) and
+// resets the counter to zero for the next call.
+//
+// Launched with programmatic dependent launch: the weight copies start before
+// the previous kernel in the stream has finished; x, y and the workspace wait
+// for it.
 #include <algorithm>
 
 #include "s12_device.cuh"
 #include "s12_launch.h"
 
 namespace s12 {
+namespace gemv {
 
-constexpr int kPassTiles = 4;   // tiles per pass
-constexpr int kU = 4;           // passes whose loads are in flight together
-constexpr int kMaxWarps = 32;   // warps per CTA at most
+constexpr int kRowsPerGroup = 16;
+constexpr int kSlotFloats = 128;  // one partial: 32 lanes x 4 accumulators
+#ifndef S12_GEMV_WARPS
+#define S12_GEMV_WARPS 16
+#endif
+constexpr int kWarps = S12_GEMV_WARPS;  // warps per CTA, one CTA per SM
+constexpr int kMaxStages = 4;
+constexpr int kMaxProblems = S12_GEMV_MAX_PROBLEMS;
+constexpr uint32_t kRawBytes = 16 * 128;   // raw plane of one block
+constexpr uint32_t kCodeBytes = 16 * 64;   // code plane of one block
+constexpr uint32_t kStageBytes = kRawBytes + kCodeBytes;
+constexpr uint32_t kRingOff = 1024;        // rings start 1024-aligned (128-byte swizzle atom)
 
-struct GemvParams {
-    const uint8_t *__restrict__ raw;
-    const uint8_t *__restrict__ code;
-    const uint8_t *__restrict__ base;
-    const uint32_t *__restrict__ esc_off;
-    const uint16_t *__restrict__ esc;
+// One matrix of a grouped call.
+struct __align__(64) Problem {
+    CUtensorMap tm_raw;   // u8 [R][K], box 128 x 16, 128-byte swizzle
+    CUtensorMap tm_code;  // u8 [R][K/2], box 64 x 16
+    const uint8_t *base;
+    const uint32_t *esc_off;
+    const uint16_t *esc;
+    const uint16_t *x;    // B x K bf16
+    float *y;             // B x R fp32
     uint64_t n_esc;
-    const uint16_t *__restrict__ x;
-    float *__restrict__ y;
+    long long block0;     // first block of this matrix in the grouped numbering
+    int R, K, T, n_groups;
+    int group0;           // first row group of this matrix in the grouped numbering
+};
+
+struct __align__(64) Params {
+    Problem prob[kMaxProblems];
     uint32_t *err;
-    int R, K, T, SPR;  // rows, columns, tiles per row, passes per row
-    int NW;            // warps per CTA
-    int x_smem;        // 1: x staged in shared memory
-    uint32_t x_off, part_off;
+    float *part;    // workspace: [n_units][2][kSlotFloats] partials
+    uint32_t *cnt;  // workspace: one arrival counter per row group (zero between calls)
+    long long n_blocks;
+    int n_problems, B;
+    int n_units;    // warps in the grid
+    int stages;     // ring depth per warp, 2..kMaxStages
 };
-
-// Boundary partial sums: the first and last rows of a warp's range that
-// other warps share.
-template <int B>
-struct Part {
-    int row[2];
-    float v[2][B];
-};
-
-// Consumer warps per CTA for batch B: enough warps to hide the HBM latency
-// within the register budget of the batch's accumulators.
-template <int B>
-constexpr int warps_for_batch() {
-    return B == 1 ? 32 : (B <= 3 ? 16 : 8);
-}
-
-// acc0 += lo(w) * lo(x), acc1 += hi(w) * hi(x): BF16 operands, FP32 accumulate.
-__device__ __forceinline__ void fma_bf16x2(float &acc0, float &acc1, uint32_t w, uint32_t x) {
-    asm("{\n\t.reg .b16 wl, wh, xl, xh;\n\t"
-        "mov.b32 {wl, wh}, %2;\n\t"
-        "mov.b32 {xl, xh}, %3;\n\t"
-        "fma.rn.f32.bf16 %0, wl, xl, %0;\n\t"
-        "fma.rn.f32.bf16 %1, wh, xh, %1;\n\t}"
-        : "+f"(acc0), "+f"(acc1)
-        : "r"(w), "r"(x));
-}
 
 __device__ __forceinline__ uint4 lds128(uint32_t a) {
     uint4 v;
@@ -93,193 +97,422 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
     return v;
 }
 
-// A position in this CTA's pass sequence: CTA-relative row and pass in row.
-struct PassPos {
-    int r, j;
+// d += A * B for one m16n8k16 product, BF16 operands, FP32 accumulators.
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mbar_init_s(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx_s(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+// Wait for phase `parity` of the barrier; false after about a second.
+__device__ __forceinline__ bool mbar_wait_s(uint32_t bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity))
+        if (clock64() - t0 > kWaitCycles) return false;
+    return true;
+}
+
+// 2-D TMA copy of one box into this CTA's shared memory, completing on bar.
+__device__ __forceinline__ void tma2d(uint32_t dst, const CUtensorMap *tm, int c0, int c1, uint32_t bar,
+                                      uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+        "l"(tm), "r"(c0), "r"(c1), "r"(bar), "l"(policy)
+        : "memory");
+}
+
+// Position of a block: matrix, 16-row group and tile column.
+struct Pos {
+    int p, grp, j;
 };
 
-template <int B>
-__global__ void __launch_bounds__(32 * warps_for_batch<B>(), 1) gemv_kernel(const __grid_constant__ GemvParams p) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int R = p.R, K = p.K, T = p.T, SPR = p.SPR, NW = p.NW;
-    const int r0 = static_cast<int>(static_cast<int64_t>(blockIdx.x) * R / gridDim.x);
-    const int r1 = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * R / gridDim.x);
-    const int n_pass = (r1 - r0) * SPR;
-    // this warp's passes [pa, pb)
-    const int pa = static_cast<int>(static_cast<int64_t>(warp) * n_pass / NW);
-    const int pb = static_cast<int>(static_cast<int64_t>(warp + 1) * n_pass / NW);
-    uint64_t *xbar = reinterpret_cast<uint64_t *>(smem);
-    Part<B> *parts = reinterpret_cast<Part<B> *>(smem + p.part_off);
-
-    if (threadIdx.x == 0) {
-        mbar_init(xbar, 1);
-        fence_barrier_init();
-        grid_launch_dependents();
-    }
-    if (lane == 0) parts[warp].row[0] = parts[warp].row[1] = -1;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        grid_dependency_wait();  // x may be written by the previous kernel in the stream
-        if (p.x_smem) {
-            mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(B * K * 2));
-            for (int b = 0; b < B; ++b)
-                tma_load_1d(smem + p.x_off + static_cast<size_t>(b) * K * 2, p.x + static_cast<size_t>(b) * K,
-                            static_cast<uint32_t>(K * 2), xbar, policy_evict_last());
-        } else {
-            mbar_arrive(xbar);
+__device__ __forceinline__ void advance(Pos &ps, const Params &pr) {
+    if (++ps.j == pr.prob[ps.p].T) {
+        ps.j = 0;
+        if (++ps.grp == pr.prob[ps.p].n_groups) {
+            ps.grp = 0;
+            ++ps.p;
         }
-    }
-    const bool x_ok = mbar_wait(xbar, 0, p.err);
-    grid_dependency_wait();  // y may be read by earlier kernels
-
-    const uint32_t g = static_cast<uint32_t>(lane >> 3);         // tile of the pass this lane decodes
-    const uint32_t wofs = static_cast<uint32_t>(lane & 7) * 16;  // first weight of the lane in its tile
-    const uint32_t x_lane = smem_addr(smem + p.x_off) + (g * 128 + wofs) * 2;  // lane's x in pass 0 of a row
-    const uint16_t *xg_lane = p.x + g * 128 + wofs;
-    const bool check = p.err != nullptr;
-
-    float acc[B][2];  // running partial of row cur_rr
-#pragma unroll
-    for (int b = 0; b < B; ++b) acc[b][0] = acc[b][1] = 0.f;
-    PassPos q = {pa / SPR, pa - (pa / SPR) * SPR};  // next pass
-    int cur_rr = q.r;
-
-    auto flush = [&](int rr) {  // reduce this warp's partial of CTA row rr and publish it
-        float v[B];
-#pragma unroll
-        for (int b = 0; b < B; ++b) {
-            float t = acc[b][0] + acc[b][1];
-#pragma unroll
-            for (int d = 16; d > 0; d >>= 1) t += __shfl_xor_sync(0xFFFFFFFFu, t, d);
-            v[b] = t;
-            acc[b][0] = acc[b][1] = 0.f;
-        }
-        if (lane == 0) {
-            const bool starts_before = rr * SPR < pa, ends_after = (rr + 1) * SPR > pb;
-            if (!starts_before && !ends_after) {
-#pragma unroll
-                for (int b = 0; b < B; ++b) p.y[static_cast<size_t>(b) * R + r0 + rr] = v[b];
-            } else {
-                const int e = starts_before ? 0 : 1;
-                parts[warp].row[e] = rr;
-#pragma unroll
-                for (int b = 0; b < B; ++b) parts[warp].v[e][b] = v[b];
-            }
-        }
-    };
-
-    for (int P0 = pa; P0 < pb && x_ok; P0 += kU) {
-        // positions of the U passes
-        PassPos qp[kU];
-        qp[0] = q;
-#pragma unroll
-        for (int i = 1; i < kU; ++i) {
-            qp[i] = qp[i - 1];
-            if (++qp[i].j == SPR) {
-                qp[i].j = 0;
-                ++qp[i].r;
-            }
-        }
-        // issue every load of the U passes first
-        uint4 raw[kU];
-        uint2 code[kU];
-        uint32_t bse[kU], lo[kU], hi[kU];
-        bool act[kU];
-#pragma unroll
-        for (int i = 0; i < kU; ++i) {
-            const int tcol = kPassTiles * qp[i].j + static_cast<int>(g);
-            act[i] = (P0 + i < pb) && (tcol < T);
-            raw[i] = make_uint4(0, 0, 0, 0);
-            code[i] = make_uint2(0, 0);
-            bse[i] = lo[i] = hi[i] = 0;
-            if (act[i]) {
-                const uint64_t t = static_cast<uint64_t>(r0 + qp[i].r) * T + tcol;
-                raw[i] = __ldcs(reinterpret_cast<const uint4 *>(p.raw + t * 128 + wofs));
-                code[i] = __ldcs(reinterpret_cast<const uint2 *>(p.code + t * 64 + wofs / 2));
-                bse[i] = __ldg(p.base + t);
-                lo[i] = __ldg(p.esc_off + t);
-                hi[i] = __ldg(p.esc_off + t + 1);
-            }
-        }
-        float accp[kU][B][2];
-#pragma unroll
-        for (int i = 0; i < kU; ++i) {
-#pragma unroll
-            for (int b = 0; b < B; ++b) accp[i][b][0] = accp[i][b][1] = 0.f;
-            const uint32_t col_off = static_cast<uint32_t>(kPassTiles * qp[i].j) * 256u;  // bytes of x before the pass
-            uint32_t xv[B][8];
-#pragma unroll
-            for (int b = 0; b < B; ++b) {
-                uint4 a = make_uint4(0, 0, 0, 0), a2 = make_uint4(0, 0, 0, 0);
-                if (act[i]) {
-                    if (p.x_smem) {
-                        const uint32_t xa = x_lane + col_off + static_cast<uint32_t>(b * K) * 2;
-                        a = lds128(xa);
-                        a2 = lds128(xa + 16);
-                    } else {
-                        const uint4 *xp = reinterpret_cast<const uint4 *>(xg_lane + col_off / 2 + static_cast<size_t>(b) * K);
-                        a = __ldg(xp);
-                        a2 = __ldg(xp + 1);
-                    }
-                }
-                xv[b][0] = a.x; xv[b][1] = a.y; xv[b][2] = a.z; xv[b][3] = a.w;
-                xv[b][4] = a2.x; xv[b][5] = a2.y; xv[b][6] = a2.z; xv[b][7] = a2.w;
-            }
-            const uint32_t B4 = bse[i] * 0x01010101u;
-            uint32_t w[8];
-            decode16(raw[i], code[i], B4, w);
-            const uint32_t m0 = escape_nibbles(code[i].x), m1 = escape_nibbles(code[i].y);
-            if (check && bse[i] > kMaxBase) raise_flag(p.err, S12_FLAG_BASE);
-            if (__ballot_sync(0xFFFFFFFFu, (m0 | m1) != 0 || lo[i] != hi[i]))
-                fix_escapes(w, raw[i], code[i], B4, m0, m1, lo[i], hi[i], act[i], p.n_esc, p.esc, p.err);
-#pragma unroll
-            for (int qq = 0; qq < 8; ++qq)
-#pragma unroll
-                for (int b = 0; b < B; ++b) fma_bf16x2(accp[i][b][0], accp[i][b][1], w[qq], xv[b][qq]);
-        }
-        // fold the passes into rows
-#pragma unroll
-        for (int i = 0; i < kU; ++i) {
-            if (P0 + i < pb) {
-                if (qp[i].r != cur_rr) {
-                    flush(cur_rr);
-                    cur_rr = qp[i].r;
-                }
-#pragma unroll
-                for (int b = 0; b < B; ++b) {
-                    acc[b][0] += accp[i][b][0];
-                    acc[b][1] += accp[i][b][1];
-                }
-            }
-        }
-        q = qp[kU - 1];
-        if (++q.j == SPR) {
-            q.j = 0;
-            ++q.r;
-        }
-    }
-    if (x_ok && pa < pb) flush(cur_rr);
-    __syncthreads();
-    // rows shared by neighbouring warps: sum the partials in warp order
-    if (warp == 0 && lane < B) {
-        int row = -1;
-        float sum = 0.f;
-        for (int w = 0; w < NW; ++w) {
-            for (int e = 0; e < 2; ++e) {
-                const int rr = parts[w].row[e];
-                if (rr < 0) continue;
-                if (rr != row) {
-                    if (row >= 0) p.y[static_cast<size_t>(lane) * R + r0 + row] = sum;
-                    row = rr;
-                    sum = 0.f;
-                }
-                sum += parts[w].v[e][lane];
-            }
-        }
-        if (row >= 0) p.y[static_cast<size_t>(lane) * R + r0 + row] = sum;
     }
 }
+
+// Position of grouped block b (b < n_blocks).
+__device__ __forceinline__ Pos locate(const Params &pr, long long b) {
+    int p = 0;
+    while (p + 1 < pr.n_problems && pr.prob[p + 1].block0 <= b) ++p;
+    const long long local = b - pr.prob[p].block0;
+    const int T = pr.prob[p].T;
+    return Pos{p, static_cast<int>(local / T), static_cast<int>(local % T)};
+}
+
+// Grouped row-group index of a position (the arrival-counter index).
+__device__ __forceinline__ long long group_id(const Params &pr, Pos ps) { return pr.prob[ps.p].group0 + ps.grp; }
+
+// Per-tile metadata of the lane's two rows for one block.
+struct Meta {
+    uint32_t baseA, baseB, loA, hiA, loB, hiB;
+};
+
+// Rows past the end (the TMA copies read them as zeros) read the last row's
+// metadata but report no escapes.
+__device__ __forceinline__ Meta load_meta(const Problem &m_, Pos ps, int g) {
+    const int rA = ps.grp * kRowsPerGroup + g, rB = rA + 8;
+    const size_t tA = static_cast<size_t>(min(rA, m_.R - 1)) * m_.T + ps.j;
+    const size_t tB = static_cast<size_t>(min(rB, m_.R - 1)) * m_.T + ps.j;
+    Meta m;
+    m.baseA = __ldg(m_.base + tA);
+    m.baseB = __ldg(m_.base + tB);
+    m.loA = __ldg(m_.esc_off + tA);
+    m.hiA = __ldg(m_.esc_off + tA + 1);
+    m.loB = __ldg(m_.esc_off + tB);
+    m.hiB = __ldg(m_.esc_off + tB + 1);
+    if (rA >= m_.R) m.hiA = m.loA;
+    if (rB >= m_.R) m.hiB = m.loB;
+    return m;
+}
+
+// The first escape value of a tile with escapes (0 otherwise), fetched ahead
+// of its use.
+__device__ __forceinline__ uint32_t first_escape(const Problem &m_, uint32_t lo, uint32_t hi) {
+    uint32_t v = 0;
+    if (lo < hi && lo < m_.n_esc) v = __ldg(m_.esc + lo);
+    return v;
+}
+
+// First block of warp unit u's range.
+__device__ __forceinline__ long long unit_start(long long u, long long n_blocks, int n_units) {
+    return u * n_blocks / n_units;
+}
+
+__device__ __forceinline__ long long unit_of_block(long long b, long long n, int nu) {
+    return ((b + 1) * nu + n - 1) / n - 1;
+}
+
+}  // namespace gemv
+}  // namespace s12
+
+namespace s12 {
+namespace gemv {
+
+// Write the accumulators of row group `grp` of matrix m to its y: lane
+// (g, q) holds D[g][2q], D[g][2q+1], D[g+8][2q], D[g+8][2q+1] (row of W,
+// batch row).
+__device__ __forceinline__ void store_y(const Problem &m, int B, const float (&a)[4], int grp, int g, int q) {
+    const int rA = grp * kRowsPerGroup + g;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = rA + (i >= 2 ? 8 : 0);
+        const int b = 2 * q + (i & 1);
+        if (r < m.R && b < B) m.y[static_cast<size_t>(b) * m.R + r] = a[i];
+    }
+}
+
+// The warp's accumulators of the row group at `ps` are complete for its part
+// of the group: store them, or hand them to the stream-K fix-up.  G0 is the
+// grouped index of the warp's first row group.
+__device__ __noinline__ void finish_group(const Params &pr, float4 a4, Pos ps, long long u, long long ub0,
+                                          long long ub1, long long G0, int lane) {
+    const float acc[4] = {a4.x, a4.y, a4.z, a4.w};
+    const int g = lane >> 2, q = lane & 3;
+    const Problem &m = pr.prob[ps.p];
+    const long long n = pr.n_blocks;
+    const long long gb0 = m.block0 + static_cast<long long>(ps.grp) * m.T, gb1 = gb0 + m.T;
+    if (gb0 >= ub0 && gb1 <= ub1) {
+        store_y(m, pr.B, acc, ps.grp, g, q);
+        return;
+    }
+    const long long G = m.group0 + ps.grp;
+    const int slot = G == G0 ? 0 : 1;
+    float4 *mine = reinterpret_cast<float4 *>(pr.part + (static_cast<size_t>(u) * 2 + slot) * kSlotFloats) + lane;
+    __stcg(mine, a4);
+    __threadfence();
+    __syncwarp();
+    const long long uf = unit_of_block(gb0, n, pr.n_units), ul = unit_of_block(gb1 - 1, n, pr.n_units);
+    uint32_t n_contrib = 0;
+    for (long long v = uf; v <= ul; ++v)
+        if (unit_start(v, n, pr.n_units) < unit_start(v + 1, n, pr.n_units)) ++n_contrib;
+    uint32_t prev = 0;
+    if (lane == 0) prev = atomicAdd(pr.cnt + G, 1u);
+    prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
+    if (prev + 1 != n_contrib) return;
+    __threadfence();
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
+    for (long long v = uf; v <= ul; ++v) {
+        const long long vs = unit_start(v, n, pr.n_units);
+        if (vs >= unit_start(v + 1, n, pr.n_units)) continue;
+        const int sl = group_id(pr, locate(pr, vs)) == G ? 0 : 1;
+        const float4 t =
+            __ldcg(reinterpret_cast<const float4 *>(pr.part + (static_cast<size_t>(v) * 2 + sl) * kSlotFloats) + lane);
+        s[0] += t.x;
+        s[1] += t.y;
+        s[2] += t.z;
+        s[3] += t.w;
+    }
+    store_y(m, pr.B, s, ps.grp, g, q);
+    if (lane == 0) atomicExch(pr.cnt + G, 0u);
+}
+
+// Escapes of one tile row for this lane (set up only for rows whose tile has
+// escapes): the escape-nibble masks of the lane's two chunks, the stream
+// index of each chunk's first escape, the end of the tile's escapes, and the
+// tile's first escape (index and prefetched value).
+struct EscRow {
+    uint2 m0, m1;
+    uint32_t s0, s1, limit, first, first_val;
+};
+
+__device__ __forceinline__ uint32_t count2(uint2 m) { return __popc(m.x) + __popc(m.y); }
+
+// Called by whole quads (the lanes of `quads`, a union of complete quads that
+// share a tile row).  Chunk order within a tile row: lane q = 0..3, half 0
+// then half 1 (chunk 2q + h covers columns 32q + 16h .. +15).  The tile's
+// code-15 count is checked against its esc_off span.
+__device__ __forceinline__ void prepare_row(uint4 c, uint32_t lo, uint32_t hi, uint32_t fv, uint64_t n_esc,
+                                            uint32_t *err, unsigned quads, int q, EscRow &e) {
+    e.m0 = make_uint2(escape_nibbles(c.x), escape_nibbles(c.y));
+    e.m1 = make_uint2(escape_nibbles(c.z), escape_nibbles(c.w));
+    const uint32_t n0 = count2(e.m0), n = n0 + count2(e.m1);
+    uint32_t incl = n;
+#pragma unroll
+    for (int d = 1; d < 4; d <<= 1) {
+        const uint32_t v = __shfl_up_sync(quads, incl, d, 4);
+        if (q >= d) incl += v;
+    }
+    const uint32_t tot = __shfl_sync(quads, incl, 3, 4);
+    e.s0 = lo + incl - n;
+    e.s1 = e.s0 + n0;
+    e.limit = lo <= hi ? static_cast<uint32_t>(hi < n_esc ? hi : n_esc) : 0u;
+    e.first = lo;
+    e.first_val = fv;
+    if (q == 0 && tot != hi - lo) raise_flag(err, S12_FLAG_ESC_COUNT);
+}
+
+// A chunk with escapes: decode it again with the escape nibbles cleared (so
+// base + code never carries out of a byte, even for base 241), then put the
+// exact value of each escaped weight in place, reading the stream from
+// index `idx`; reads at or past the tile's end are skipped and flagged.
+__device__ __forceinline__ void fix_chunk(uint32_t (&w)[8], uint4 raw, uint2 code, uint32_t base, uint2 m,
+                                          uint32_t idx, const EscRow &e, const uint16_t *__restrict__ esc,
+                                          uint32_t *err) {
+    decode16(raw, make_uint2(clear_escapes(code.x, m.x), clear_escapes(code.y, m.y)), base * 0x01010101u, w);
+    uint32_t m0 = m.x, m1 = m.y;
+    while (m0 | m1) {
+        int j;
+        if (m0) {
+            j = (__ffs(m0) - 1) >> 2;
+            m0 &= m0 - 1;
+        } else {
+            j = 8 + ((__ffs(m1) - 1) >> 2);
+            m1 &= m1 - 1;
+        }
+        uint32_t v = 0;
+        if (idx < e.limit)
+            v = idx == e.first ? e.first_val : __ldg(esc + idx);
+        else
+            raise_flag(err, S12_FLAG_ESC_RANGE);
+        ++idx;
+        const int r = j >> 1;
+        const uint32_t keep = (j & 1) ? 0x0000FFFFu : 0xFFFF0000u;
+        const uint32_t put = (j & 1) ? (v << 16) : v;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (i == r) w[i] = (w[i] & keep) | put;
+    }
+}
+
+__device__ __forceinline__ float4 sum_halves(const float (&acc)[2][4]) {
+    return make_float4(acc[0][0] + acc[1][0], acc[0][1] + acc[1][1], acc[0][2] + acc[1][2], acc[0][3] + acc[1][3]);
+}
+
+// The lane's 16 activations (batch row gx, columns j*128 + 32q + 16h ..),
+// read through the L1 cache.
+__device__ __forceinline__ void load_x(uint32_t (&xw)[8], const uint16_t *xl, int j, int h) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(xl + static_cast<size_t>(j) * kTile + h * 16);
+    const uint4 a = __ldg(src), b = __ldg(src + 1);
+    xw[0] = a.x; xw[1] = a.y; xw[2] = a.z; xw[3] = a.w;
+    xw[4] = b.x; xw[5] = b.y; xw[6] = b.z; xw[7] = b.w;
+}
+
+// One half of a block: four m16n8k16 products of rows g / g+8 with x.
+__device__ __forceinline__ void half_mma(float (&acc)[4], const uint32_t (&wa)[8], const uint32_t (&wb)[8],
+                                         const uint32_t (&xw)[8]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) mma16816(acc, wa[2 * i], wb[2 * i], wa[2 * i + 1], wb[2 * i + 1], xw[2 * i], xw[2 * i + 1]);
+}
+
+}  // namespace gemv
+}  // namespace s12
+
+namespace s12 {
+namespace gemv {
+
+// Start the copies of the block at `ps` into stage st (completing on bar).
+__device__ __forceinline__ void copy_block(const Params &pr, Pos ps, uint32_t st, uint32_t bar, uint64_t pol) {
+    const Problem &m = pr.prob[ps.p];
+    mbar_expect_tx_s(bar, kStageBytes);
+    tma2d(st, &m.tm_raw, ps.j * 128, ps.grp * kRowsPerGroup, bar, pol);
+    tma2d(st + kRawBytes, &m.tm_code, ps.j * 64, ps.grp * kRowsPerGroup, bar, pol);
+}
+
+template <bool CHECK>
+__global__ void __launch_bounds__(kWarps * 32, 1) gemv_tma_kernel(const __grid_constant__ Params pr) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t sb = (smem_addr(smem_raw) + 1023u) & ~1023u;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, q = lane & 3;
+    const long long n = pr.n_blocks;
+    const long long u = static_cast<long long>(blockIdx.x) * kWarps + warp;
+    const long long ub0 = unit_start(u, n, pr.n_units), ub1 = unit_start(u + 1, n, pr.n_units);
+    const int nb = static_cast<int>(ub1 - ub0);
+    const int S = pr.stages;
+    const uint32_t bars = sb + static_cast<uint32_t>(warp) * kMaxStages * 8u;
+    const uint32_t ring = sb + kRingOff + static_cast<uint32_t>(warp * S) * kStageBytes;
+    if (threadIdx.x == 0) grid_launch_dependents();
+
+    // The weights are never written by other kernels: start the copies
+    // before waiting for the previous grid.
+    const Pos p0 = nb > 0 ? locate(pr, ub0) : Pos{0, 0, 0};
+    Pos pi = p0;  // next block to copy
+    uint64_t pol = 0;
+    if (lane == 0) {
+        pol = policy_evict_first();
+        for (int s = 0; s < S; ++s) mbar_init_s(bars + 8u * s, 1);
+        fence_barrier_init();
+        for (int s = 0; s < S && s < nb; ++s) {
+            copy_block(pr, pi, ring + s * kStageBytes, bars + 8u * s, pol);
+            advance(pi, pr);
+        }
+    }
+    __syncwarp();
+    if (nb == 0) return;
+    grid_dependency_wait();  // x, y and the workspace may belong to earlier kernels
+    const int gx = g < pr.B ? g : 0;  // batch rows past B repeat row 0; their outputs are dropped
+    // lane's shared-memory offsets inside a stage (raw rows are 128-byte swizzled)
+    const uint32_t oA0 = g * 128 + (((2 * q) ^ g) << 4), oA1 = g * 128 + (((2 * q + 1) ^ g) << 4);
+    const uint32_t oB0 = oA0 + 8 * 128, oB1 = oA1 + 8 * 128;
+    const uint32_t oCA = kRawBytes + g * 64 + 16 * q, oCB = oCA + 8 * 64;
+
+    Pos pc = p0;  // block being computed
+    Pos pn = p0;  // block whose first escapes are fetched (one ahead)
+    Pos pm = p0;  // block whose metadata is loaded (two ahead)
+    Meta m0 = load_meta(pr.prob[pm.p], pm, g), m1 = m0;
+    advance(pm, pr);
+    if (nb > 1) m1 = load_meta(pr.prob[pm.p], pm, g);
+    uint32_t fvA = first_escape(pr.prob[p0.p], m0.loA, m0.hiA), fvB = first_escape(pr.prob[p0.p], m0.loB, m0.hiB);
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};  // one chain per half
+    Pos cur = p0;
+    const long long G0 = group_id(pr, p0);
+    int s = 0;
+    uint32_t parity = 0;
+    bool ok = true;
+    for (int i = 0; i < nb; ++i) {
+        // metadata two blocks ahead, the next block's first escapes one ahead
+        Meta m2 = m1;
+        if (i + 2 < nb) {
+            advance(pm, pr);
+            m2 = load_meta(pr.prob[pm.p], pm, g);
+        }
+        uint32_t nfvA = 0, nfvB = 0;
+        if (i + 1 < nb) {
+            advance(pn, pr);  // now the position of block i + 1
+            const Problem &mn = pr.prob[pn.p];
+            nfvA = first_escape(mn, m1.loA, m1.hiA);
+            nfvB = first_escape(mn, m1.loB, m1.hiB);
+        }
+        if (pc.grp != cur.grp || pc.p != cur.p) {
+            finish_group(pr, sum_halves(acc), cur, u, ub0, ub1, G0, lane);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) acc[0][k] = acc[1][k] = 0.f;
+            cur = pc;
+        }
+        const Problem &mp = pr.prob[pc.p];
+        const uint32_t bar = bars + 8u * s;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait_s(bar, parity))) {
+            raise_flag(pr.err, S12_FLAG_TIMEOUT);
+            ok = false;
+            break;
+        }
+        const uint32_t st = ring + s * kStageBytes;
+        const uint4 rA0 = lds128(st + oA0), rA1 = lds128(st + oA1), rB0 = lds128(st + oB0), rB1 = lds128(st + oB1);
+        const uint4 cA = lds128(st + oCA), cB = lds128(st + oCB);
+        // the stage is in registers: hand it back to the copy engine
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0 && i + S < nb) copy_block(pr, pi, st, bar, pol);
+        if (i + S < nb) advance(pi, pr);
+
+        bool escA = m0.loA != m0.hiA, escB = m0.loB != m0.hiB;
+        if (CHECK) {
+            escA = escA || (escape_nibbles(cA.x) | escape_nibbles(cA.y) | escape_nibbles(cA.z) | escape_nibbles(cA.w));
+            escB = escB || (escape_nibbles(cB.x) | escape_nibbles(cB.y) | escape_nibbles(cB.z) | escape_nibbles(cB.w));
+            if (m0.baseA > static_cast<uint32_t>(kMaxBase) || m0.baseB > static_cast<uint32_t>(kMaxBase))
+                raise_flag(pr.err, S12_FLAG_BASE);
+        }
+        const unsigned qA = __ballot_sync(0xFFFFFFFFu, escA), qB = __ballot_sync(0xFFFFFFFFu, escB);
+        const bool any = (qA | qB) != 0;
+        EscRow eA, eB;
+        if (any) {
+            if (escA) prepare_row(cA, m0.loA, m0.hiA, fvA, mp.n_esc, pr.err, qA, q, eA);
+            if (escB) prepare_row(cB, m0.loB, m0.hiB, fvB, mp.n_esc, pr.err, qB, q, eB);
+        }
+        const uint32_t B4A = m0.baseA * 0x01010101u, B4B = m0.baseB * 0x01010101u;
+        const uint16_t *xl = mp.x + static_cast<size_t>(gx) * mp.K + 32 * q;
+        uint32_t xw[8], wa[8], wb[8];
+        // half 0
+        load_x(xw, xl, pc.j, 0);
+        decode16(rA0, make_uint2(cA.x, cA.y), B4A, wa);
+        decode16(rB0, make_uint2(cB.x, cB.y), B4B, wb);
+        if (any) {
+            if (escA && (eA.m0.x | eA.m0.y))
+                fix_chunk(wa, rA0, make_uint2(cA.x, cA.y), m0.baseA, eA.m0, eA.s0, eA, mp.esc, pr.err);
+            if (escB && (eB.m0.x | eB.m0.y))
+                fix_chunk(wb, rB0, make_uint2(cB.x, cB.y), m0.baseB, eB.m0, eB.s0, eB, mp.esc, pr.err);
+        }
+        half_mma(acc[0], wa, wb, xw);
+        // half 1
+        load_x(xw, xl, pc.j, 1);
+        decode16(rA1, make_uint2(cA.z, cA.w), B4A, wa);
+        decode16(rB1, make_uint2(cB.z, cB.w), B4B, wb);
+        if (any) {
+            if (escA && (eA.m1.x | eA.m1.y))
+                fix_chunk(wa, rA1, make_uint2(cA.z, cA.w), m0.baseA, eA.m1, eA.s1, eA, mp.esc, pr.err);
+            if (escB && (eB.m1.x | eB.m1.y))
+                fix_chunk(wb, rB1, make_uint2(cB.z, cB.w), m0.baseB, eB.m1, eB.s1, eB, mp.esc, pr.err);
+        }
+        half_mma(acc[1], wa, wb, xw);
+
+        advance(pc, pr);
+        m0 = m1;
+        m1 = m2;
+        fvA = nfvA;
+        fvB = nfvB;
+        if (++s == S) {
+            s = 0;
+            parity ^= 1u;
+        }
+    }
+    if (ok) {
+        finish_group(pr, sum_halves(acc), cur, u, ub0, ub1, G0, lane);
+    } else if (lane == 0) {
+        // a wait gave up: let the copies still in flight land before exiting
+        for (int k = 0; k < S; ++k) mbar_wait_s(bars + 8u * k, parity ^ (k < s ? 1u : 0u));
+    }
+}
+
+}  // namespace gemv
 
 // ---------------------------------------------------------------------------
 // Host side.
@@ -288,34 +521,77 @@ namespace {
 
 constexpr uint32_t kSmemLimit = 227 * 1024;
 
-template <int B>
-cudaError_t run(const s12_view *v, const uint16_t *x, float *y, uint32_t *err, int sms, cudaStream_t stream) {
-    GemvParams p;
-    p.raw = v->raw;
-    p.code = v->code;
-    p.base = v->base;
-    p.esc_off = v->esc_off;
-    p.esc = v->esc;
-    p.n_esc = v->n_esc;
-    p.x = x;
-    p.y = y;
-    p.err = err;
-    p.R = static_cast<int>(v->rows);
-    p.K = static_cast<int>(v->cols);
-    p.T = p.K / kTile;
-    p.SPR = (p.T + kPassTiles - 1) / kPassTiles;
-    p.NW = warps_for_batch<B>();
-    p.part_off = 128;
-    p.x_off = static_cast<uint32_t>(align_up(p.part_off + sizeof(Part<B>) * kMaxWarps, 128));
-    const uint64_t xbytes = static_cast<uint64_t>(B) * p.K * 2;
-    p.x_smem = (p.x_off + xbytes <= kSmemLimit) ? 1 : 0;
-    const uint32_t smem = p.x_off + (p.x_smem ? static_cast<uint32_t>(xbytes) : 0);
-    auto kern = gemv_kernel<B>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
+struct Plan {
+    long long n_blocks, n_groups;
+    int grid, n_units;
+    size_t part_bytes, cnt_bytes;
+};
+
+Plan plan(const s12_view *views, int count, int sms) {
+    Plan pl;
+    pl.n_blocks = pl.n_groups = 0;
+    for (int i = 0; i < count; ++i) {
+        const long long groups =
+            static_cast<long long>((views[i].rows + gemv::kRowsPerGroup - 1) / gemv::kRowsPerGroup);
+        pl.n_groups += groups;
+        pl.n_blocks += groups * static_cast<long long>(views[i].cols / kTile);
+    }
+    const long long want = (pl.n_blocks + gemv::kWarps - 1) / gemv::kWarps;
+    pl.grid = static_cast<int>(std::max(1LL, std::min<long long>(sms, want)));
+    pl.n_units = pl.grid * gemv::kWarps;
+    // sized for the largest grid so one workspace fits every call on the device
+    pl.part_bytes =
+        align_up(static_cast<uint64_t>(sms) * gemv::kWarps * 2 * gemv::kSlotFloats * sizeof(float), kAlign);
+    pl.cnt_bytes = align_up(static_cast<uint64_t>(pl.n_groups) * sizeof(uint32_t), kAlign);
+    return pl;
+}
+
+template <bool CHECK>
+int run(const s12_view *views, int count, const uint16_t *const *x, int B, float *const *y, void *ws,
+        uint32_t *err, const Plan &pl, cudaStream_t stream) {
+    gemv::Params pr = {};
+    long long block0 = 0;
+    int group0 = 0;
+    for (int i = 0; i < count; ++i) {
+        const s12_view *v = views + i;
+        gemv::Problem &m = pr.prob[i];
+        const uint64_t R = v->rows, K = v->cols;
+        if (make_tmap_u8_2d(&m.tm_raw, v->raw, K, R, K, 128, gemv::kRowsPerGroup, true) != S12_OK)
+            return S12_ERR_CUDA;
+        if (make_tmap_u8_2d(&m.tm_code, v->code, K / 2, R, K / 2, 64, gemv::kRowsPerGroup, false) != S12_OK)
+            return S12_ERR_CUDA;
+        m.base = v->base;
+        m.esc_off = v->esc_off;
+        m.esc = v->esc;
+        m.x = x[i];
+        m.y = y[i];
+        m.n_esc = v->n_esc;
+        m.R = static_cast<int>(R);
+        m.K = static_cast<int>(K);
+        m.T = m.K / kTile;
+        m.n_groups = (m.R + gemv::kRowsPerGroup - 1) / gemv::kRowsPerGroup;
+        m.block0 = block0;
+        m.group0 = group0;
+        block0 += static_cast<long long>(m.n_groups) * m.T;
+        group0 += m.n_groups;
+    }
+    pr.err = err;
+    pr.part = static_cast<float *>(ws);
+    pr.cnt = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(ws) + pl.part_bytes);
+    pr.n_blocks = pl.n_blocks;
+    pr.n_problems = count;
+    pr.B = B;
+    pr.n_units = pl.n_units;
+    pr.stages = gemv::kMaxStages;
+    // 1 KB alignment slack, barriers, then the warps' rings
+    const uint32_t smem = 1024 + gemv::kRingOff + gemv::kWarps * pr.stages * gemv::kStageBytes;
+    if (smem > kSmemLimit) return S12_ERR_CUDA;
+    auto kern = gemv::gemv_tma_kernel<CHECK>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return S12_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(std::min(sms, p.R));
-    cfg.blockDim = dim3(32 * p.NW);
+    cfg.gridDim = dim3(pl.grid);
+    cfg.blockDim = dim3(32 * gemv::kWarps);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -323,26 +599,26 @@ cudaError_t run(const s12_view *v, const uint16_t *x, float *y, uint32_t *err, i
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, p);
+    return cudaLaunchKernelEx(&cfg, kern, pr) == cudaSuccess ? S12_OK : S12_ERR_CUDA;
 }
 
 }  // namespace
 
-int launch_gemv(const s12_view *v, const uint16_t *x, int B, float *y, uint32_t *err, cudaStream_t stream) {
+size_t gemv_ws_bytes(const s12_view *views, int count) {
+    int sms = 0;
+    if (device_sms(&sms) != cudaSuccess) return 0;
+    const Plan pl = plan(views, count, sms);
+    return pl.part_bytes + pl.cnt_bytes;
+}
+
+int launch_gemv(const s12_view *views, int count, const uint16_t *const *x, int B, float *const *y, void *ws,
+                size_t ws_bytes, uint32_t *err, cudaStream_t stream) {
     int sms = 0;
     if (device_sms(&sms) != cudaSuccess) return S12_ERR_CUDA;
-    cudaError_t e;
-    switch (B) {
-        case 1: e = run<1>(v, x, y, err, sms, stream); break;
-        case 2: e = run<2>(v, x, y, err, sms, stream); break;
-        case 3: e = run<3>(v, x, y, err, sms, stream); break;
-        case 4: e = run<4>(v, x, y, err, sms, stream); break;
-        case 5: e = run<5>(v, x, y, err, sms, stream); break;
-        case 6: e = run<6>(v, x, y, err, sms, stream); break;
-        case 7: e = run<7>(v, x, y, err, sms, stream); break;
-        default: e = run<8>(v, x, y, err, sms, stream); break;
-    }
-    return e == cudaSuccess ? S12_OK : S12_ERR_CUDA;
+    const Plan pl = plan(views, count, sms);
+    if (ws_bytes < pl.part_bytes + pl.cnt_bytes) return S12_ERR_CAPACITY;
+    return err ? run<true>(views, count, x, B, y, ws, err, pl, stream)
+               : run<false>(views, count, x, B, y, ws, err, pl, stream);
 }
 
 }  // namespace s12

@@ -56,8 +56,8 @@ PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
 std::once_flag g_encode_once;
 }  // namespace
 
-int make_tmap_u64_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t rows, uint64_t row_stride,
-                     uint32_t box_inner, uint32_t box_rows) {
+int make_tmap_u8_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t rows, uint64_t row_stride,
+                    uint32_t box_inner, uint32_t box_rows, bool swizzle128) {
     std::call_once(g_encode_once, [] {
         void *fn = nullptr;
         cudaDriverEntryPointQueryResult q;
@@ -70,8 +70,9 @@ int make_tmap_u64_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_
     const cuuint64_t strides[1] = {row_stride};
     const cuuint32_t box[2] = {box_inner, box_rows};
     const cuuint32_t estr[2] = {1, 1};
-    CUresult r = g_encode_tiled(out, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<void *>(base), dims, strides, box,
-                                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+    CUresult r = g_encode_tiled(out, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box,
+                                estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? S12_OK : S12_ERR_CUDA;
 }
@@ -162,14 +163,36 @@ int s12_decode(const s12_view *v, uint16_t *out, uint32_t *err_flag, void *strea
     return launch_decode(v, out, err_flag, static_cast<cudaStream_t>(stream));
 }
 
-int s12_gemv(const s12_view *v, const uint16_t *x, int B, float *y, uint32_t *err_flag, void *stream) {
+size_t s12_gemv_ws_bytes(const s12_view *v, int B) { return s12_gemv_multi_ws_bytes(v, 1, B); }
+
+size_t s12_gemv_multi_ws_bytes(const s12_view *views, int count, int B) {
+    if (!views || count < 1 || count > S12_GEMV_MAX_PROBLEMS || B < 1 || B > S12_GEMV_MAX_BATCH) return 0;
+    for (int i = 0; i < count; ++i)
+        if (check_view(views + i) != S12_OK) return 0;
+    return gemv_ws_bytes(views, count);
+}
+
+int s12_gemv_multi(const s12_view *views, int count, const uint16_t *const *x, int B, float *const *y, void *ws,
+                   size_t ws_bytes, uint32_t *err_flag, void *stream) {
+    if (!views || !x || !y || !ws) return S12_ERR_ARG;
+    if (count < 1 || count > S12_GEMV_MAX_PROBLEMS || B < 1 || B > S12_GEMV_MAX_BATCH) return S12_ERR_SHAPE;
+    for (int i = 0; i < count; ++i) {
+        int rc = check_view(views + i);
+        if (rc != S12_OK) return rc;
+        if (!x[i] || !y[i]) return S12_ERR_ARG;
+        if (views[i].rows > 0x7FFFFFFFull || views[i].cols > 0x7FFFFFFFull) return S12_ERR_SHAPE;
+        if (!aligned16(x[i]) || !aligned4(y[i])) return S12_ERR_ALIGN;
+    }
+    if (!aligned16(ws) || (err_flag && !aligned4(err_flag))) return S12_ERR_ALIGN;
+    return launch_gemv(views, count, x, B, y, ws, ws_bytes, err_flag, static_cast<cudaStream_t>(stream));
+}
+
+int s12_gemv(const s12_view *v, const uint16_t *x, int B, float *y, void *ws, size_t ws_bytes, uint32_t *err_flag,
+             void *stream) {
+    if (!v || !x || !y || !ws) return S12_ERR_ARG;
     int rc = check_view(v);
     if (rc != S12_OK) return rc;
-    if (!x || !y) return S12_ERR_ARG;
-    if (B < 1 || B > S12_GEMV_MAX_BATCH) return S12_ERR_SHAPE;
-    if (v->rows > 0x7FFFFFFFull || v->cols > 0x7FFFFFFFull) return S12_ERR_SHAPE;
-    if (!aligned16(x) || !aligned4(y) || (err_flag && !aligned4(err_flag))) return S12_ERR_ALIGN;
-    return launch_gemv(v, x, B, y, err_flag, static_cast<cudaStream_t>(stream));
+    return s12_gemv_multi(v, 1, &x, B, &y, ws, ws_bytes, err_flag, stream);
 }
 
 size_t s12_gemm_ws_bytes(const s12_view *v, int M) {

@@ -11,14 +11,17 @@ namespace s12 {
 // Number of SMs of the current device (cached per device).
 cudaError_t device_sms(int *sms);
 
-// Tiled TMA descriptor for a row-major 2-D array of 8-byte elements:
-// `inner` elements per row, `rows` rows, `row_stride` bytes between rows,
-// box of box_inner x box_rows elements, out-of-bounds elements read as 0.
-int make_tmap_u64_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t rows, uint64_t row_stride,
-                     uint32_t box_inner, uint32_t box_rows);
+// Tiled TMA descriptor for a row-major 2-D array of bytes: `inner` bytes
+// per row, `rows` rows, `row_stride` bytes between rows (multiple of 16),
+// box of box_inner x box_rows bytes (box_inner a multiple of 16; 128 with
+// the 128-byte swizzle), out-of-bounds bytes read as 0.
+int make_tmap_u8_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t rows, uint64_t row_stride,
+                    uint32_t box_inner, uint32_t box_rows, bool swizzle128);
 
 int launch_decode(const s12_view *v, uint16_t *out, uint32_t *err, cudaStream_t stream);
-int launch_gemv(const s12_view *v, const uint16_t *x, int B, float *y, uint32_t *err, cudaStream_t stream);
+size_t gemv_ws_bytes(const s12_view *views, int count);
+int launch_gemv(const s12_view *views, int count, const uint16_t *const *x, int B, float *const *y, void *ws,
+                size_t ws_bytes, uint32_t *err, cudaStream_t stream);
 int launch_bf16_gemv(const uint16_t *w, int64_t rows, int64_t cols, const uint16_t *x, int B, float *y,
                      cudaStream_t stream);
 size_t encode_ws_bytes(int64_t rows, int64_t cols);

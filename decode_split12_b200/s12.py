@@ -34,7 +34,7 @@ S12_FLAG_TIMEOUT = 8
 
 EXPORTED = (
     "s12_error_string", "s12_device_check", "s12_container_bytes", "s12_encode_ws_bytes", "s12_encode",
-    "s12_open", "s12_decode", "s12_gemv", "s12_gemm_ws_bytes", "s12_gemm_skinny", "s12_stats_ws_bytes",
+    "s12_open", "s12_decode", "s12_gemv_ws_bytes", "s12_gemv", "s12_gemv_multi_ws_bytes", "s12_gemv_multi", "s12_gemm_ws_bytes", "s12_gemm_skinny", "s12_stats_ws_bytes",
     "s12_stats", "s12_bf16_gemv",
 )
 
@@ -90,7 +90,14 @@ def _lib() -> C.CDLL:
         lib.s12_open.restype = C.c_int
         lib.s12_decode.argtypes = [C.POINTER(View), _P, _P, _P]
         lib.s12_decode.restype = C.c_int
-        lib.s12_gemv.argtypes = [C.POINTER(View), _P, C.c_int, _P, _P, _P]
+        lib.s12_gemv_ws_bytes.argtypes = [C.POINTER(View), C.c_int]
+        lib.s12_gemv_ws_bytes.restype = _SZ
+        lib.s12_gemv.argtypes = [C.POINTER(View), _P, C.c_int, _P, _P, _SZ, _P, _P]
+        lib.s12_gemv_multi_ws_bytes.argtypes = [C.POINTER(View), C.c_int, C.c_int]
+        lib.s12_gemv_multi_ws_bytes.restype = _SZ
+        lib.s12_gemv_multi.argtypes = [C.POINTER(View), C.c_int, C.POINTER(_P), C.c_int, C.POINTER(_P), _P, _SZ, _P,
+                                       _P]
+        lib.s12_gemv_multi.restype = C.c_int
         lib.s12_gemv.restype = C.c_int
         lib.s12_gemm_ws_bytes.argtypes = [C.POINTER(View), C.c_int]
         lib.s12_gemm_ws_bytes.restype = _SZ
@@ -194,6 +201,7 @@ def s12_encode(w: torch.Tensor, ws: torch.Tensor | None = None, stream=None) -> 
 def s12_open(blob: torch.Tensor) -> View:
     v = View()
     _check(_lib().s12_open(_dptr(blob), blob.numel() * blob.element_size(), C.byref(v)), "s12_open")
+    v._blob = blob  # the view points into blob's memory: keep it alive as long as the view
     return v
 
 
@@ -205,14 +213,58 @@ def s12_decode(view: View, out: torch.Tensor | None = None, err_flag: torch.Tens
     return out
 
 
-def s12_gemv(view: View, x: torch.Tensor, y: torch.Tensor | None = None, err_flag: torch.Tensor | None = None,
-             stream=None) -> torch.Tensor:
+def s12_gemv_ws_bytes(view: View, B: int = 1) -> int:
+    return int(_lib().s12_gemv_ws_bytes(C.byref(view), B))
+
+
+def gemv_workspace(view: View, B: int = 1, device=None) -> torch.Tensor:
+    """A zero-filled workspace large enough for s12_gemv on `view`; the call
+    leaves it zero-filled, so it can be reused by later calls on one stream."""
+    need = max(s12_gemv_ws_bytes(view, B), 256)
+    return torch.zeros(need, dtype=torch.uint8, device=device or "cuda")
+
+
+def s12_gemv(view: View, x: torch.Tensor, y: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+             err_flag: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     x = _u16(x)
     B = x.shape[0] if x.dim() == 2 else 1
     if y is None:
         y = torch.empty((B, view.rows), dtype=torch.float32, device=x.device)
-    _check(_lib().s12_gemv(C.byref(view), _dptr(x), B, _dptr(y), _dptr(err_flag), _stream(stream)), "s12_gemv")
+    if ws is None:
+        ws = gemv_workspace(view, B, x.device)
+    _check(_lib().s12_gemv(C.byref(view), _dptr(x), B, _dptr(y), _dptr(ws), ws.numel(), _dptr(err_flag),
+                           _stream(stream)), "s12_gemv")
     return y
+
+
+def _view_array(views):
+    arr = (View * len(views))()
+    for i, v in enumerate(views):
+        arr[i] = v
+    return arr
+
+
+def s12_gemv_multi_ws_bytes(views, B: int = 1) -> int:
+    return int(_lib().s12_gemv_multi_ws_bytes(_view_array(views), len(views), B))
+
+
+def s12_gemv_multi(views, xs, ys=None, ws: torch.Tensor | None = None, err_flag: torch.Tensor | None = None,
+                   stream=None):
+    """Several independent fused decode-GEMVs in one launch; returns the list
+    of y tensors (allocated when `ys` is None)."""
+    xs = [_u16(x) for x in xs]
+    B = xs[0].shape[0] if xs[0].dim() == 2 else 1
+    if ys is None:
+        ys = [torch.empty((B, v.rows), dtype=torch.float32, device=xs[0].device) for v in views]
+    arr = _view_array(views)
+    if ws is None:
+        need = max(int(_lib().s12_gemv_multi_ws_bytes(arr, len(views), B)), 256)
+        ws = torch.zeros(need, dtype=torch.uint8, device=xs[0].device)
+    xp = (_P * len(xs))(*[_dptr(x) for x in xs])
+    yp = (_P * len(ys))(*[_dptr(y) for y in ys])
+    _check(_lib().s12_gemv_multi(arr, len(views), xp, B, yp, _dptr(ws), ws.numel(), _dptr(err_flag),
+                                 _stream(stream)), "s12_gemv_multi")
+    return ys
 
 
 def s12_gemm_ws_bytes(view: View, M: int) -> int:

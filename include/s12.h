@@ -80,6 +80,7 @@ extern "C" {
 
 #define S12_TILE 128
 #define S12_GEMV_MAX_BATCH 8
+#define S12_GEMV_MAX_PROBLEMS 8 /* matrices in one s12_gemv_multi call */
 #define S12_GEMM_MIN_M 16
 #define S12_GEMM_MAX_M 256
 
@@ -162,14 +163,54 @@ int s12_decode(const s12_view *v, uint16_t *out, uint32_t *err_flag, void *strea
  * decode the exact BF16 values into registers or shared memory and use them
  * at once in the matrix product) ---- */
 
+/* Workspace bytes s12_gemv needs for this container (any 1 <= B <= 8; 0
+ * for an invalid view or B).  The size depends on the row count and on the
+ * SM count of the current device, not on B, so one workspace of the largest
+ * size serves every matrix of a model on that device. */
+size_t s12_gemv_ws_bytes(const s12_view *v, int B);
+
 /* y[b][n] = sum_k W[n][k] * x[b][k] for b < B, 1 <= B <= 8.
- *   x: device BF16, B x cols row-major.   y: device FP32, B x rows
- *   row-major (4-byte alignment suffices), overwritten.
- * Weights are decoded in registers from shared-memory tiles staged by the
- * TMA engine and multiplied in FP32; the sum order is fixed, so repeated
- * calls give identical y. */
-int s12_gemv(const s12_view *v, const uint16_t *x, int B, float *y, uint32_t *err_flag,
-             void *stream);
+ *   x:  device BF16, B x cols row-major.
+ *   y:  device FP32, B x rows row-major (4-byte alignment suffices),
+ *       overwritten.
+ *   ws: device workspace of at least s12_gemv_ws_bytes(v, B) bytes (else
+ *       S12_ERR_CAPACITY), owned by the caller.  It must be ZERO-FILLED
+ *       before its first use (for instance one cudaMemsetAsync after
+ *       allocation); every call leaves it zero-filled again when it returns.
+ *       Two calls that may run at the same time (different streams) need
+ *       different workspaces.
+ * Each warp decodes 16 rows x 128 columns at a time into the registers of
+ * the warp-level tensor-core product (BF16 operands, FP32 accumulation).
+ * Rows are split across warps by contiguous ranges of such blocks; a row
+ * group shared by several warps is summed by the last of them in a fixed
+ * order, so repeated calls give identical y.
+ * With err_flag given, every tile's code-15 count is checked against its
+ * esc_off span and bases above 241 are flagged; without it only tiles whose
+ * span is non-empty are checked (slightly faster; corrupt data then gives a
+ * wrong y but never an out-of-range read). */
+int s12_gemv(const s12_view *v, const uint16_t *x, int B, float *y, void *ws, size_t ws_bytes,
+             uint32_t *err_flag, void *stream);
+
+/* Workspace bytes s12_gemv_multi needs for these `count` containers (0 for
+ * invalid arguments).  Like s12_gemv_ws_bytes it depends on the row counts
+ * and the SM count, not on B. */
+size_t s12_gemv_multi_ws_bytes(const s12_view *views, int count, int B);
+
+/* Up to S12_GEMV_MAX_PROBLEMS independent fused decode-GEMVs in ONE kernel
+ * launch: for i < count, y[i][b][n] = sum_k W_i[n][k] * x[i][b][k], b < B.
+ *   views: host array of `count` opened containers (shapes may differ).
+ *   x, y:  host arrays of `count` device pointers, laid out as in s12_gemv.
+ *   ws:    zero-filled device workspace of s12_gemv_multi_ws_bytes bytes,
+ *          left zero-filled on return (same rules as s12_gemv).
+ * The blocks of all matrices are dealt to the warps of one grid as a single
+ * range, so the launch, ramp-up and tail are paid once for the group (for
+ * instance the q, k and v projections of a decoder layer, or gate and up).
+ * Results are identical to `count` separate s12_gemv calls up to the
+ * summation order (each is within the same tolerance), and identical from
+ * call to call.  Errors as for s12_gemv; a bad entry fails the whole call
+ * before any launch. */
+int s12_gemv_multi(const s12_view *views, int count, const uint16_t *const *x, int B, float *const *y,
+                   void *ws, size_t ws_bytes, uint32_t *err_flag, void *stream);
 
 /* ---- fused decode-skinny-GEMM on tcgen05 tensor cores ---- */
 

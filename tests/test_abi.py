@@ -83,13 +83,18 @@ def test_argument_checks_need_no_device(lib):
     # an empty view
     v = s12.View()
     assert lib.s12_decode(C.byref(v), fake, None, None) == s12.S12_ERR_ARG
-    assert lib.s12_gemv(C.byref(v), fake, 1, fake, None, None) == s12.S12_ERR_ARG
+    assert lib.s12_gemv(C.byref(v), fake, 1, fake, fake, 1 << 20, None, None) == s12.S12_ERR_ARG
     # batch out of range on an otherwise well-formed view
     v.rows, v.cols, v.n_tiles = 4, 128, 4
     for f in ("container", "raw", "code", "base", "esc_off", "esc"):
         setattr(v, f, 0x100000)
-    assert lib.s12_gemv(C.byref(v), fake, 0, fake, None, None) == s12.S12_ERR_SHAPE
-    assert lib.s12_gemv(C.byref(v), fake, 9, fake, None, None) == s12.S12_ERR_SHAPE
+    assert lib.s12_gemv(C.byref(v), fake, 0, fake, fake, 1 << 20, None, None) == s12.S12_ERR_SHAPE
+    assert lib.s12_gemv(C.byref(v), fake, 9, fake, fake, 1 << 20, None, None) == s12.S12_ERR_SHAPE
+    # the GEMV workspace is mandatory and 16-byte aligned
+    assert lib.s12_gemv(C.byref(v), fake, 1, fake, None, 0, None, None) == s12.S12_ERR_ARG
+    assert lib.s12_gemv(C.byref(v), fake, 1, fake, bad, 1 << 20, None, None) == s12.S12_ERR_ALIGN
+    assert lib.s12_gemv_ws_bytes(C.byref(v), 0) == 0
+    assert lib.s12_gemv_ws_bytes(C.byref(v), 9) == 0
     assert lib.s12_gemm_skinny(C.byref(v), fake, 8, fake, fake, 1 << 20, None, None) == s12.S12_ERR_SHAPE
     assert lib.s12_gemm_skinny(C.byref(v), fake, 257, fake, fake, 1 << 20, None, None) == s12.S12_ERR_SHAPE
     assert lib.s12_open(None, 1024, C.byref(v)) == s12.S12_ERR_ARG

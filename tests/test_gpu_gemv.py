@@ -17,27 +17,36 @@ def s12(cuda_ok):
     return mod
 
 
-def _gemv(s12, w, x, flag=None):
+def _gemv(s12, w, x, flag=None, ws=None):
     blob = s12.s12_encode(to_dev(w))
     view = s12.s12_open(blob)
-    y = s12.s12_gemv(view, to_dev(x), err_flag=flag)
+    y = s12.s12_gemv(view, to_dev(x), ws=ws, err_flag=flag)
     torch.cuda.synchronize()
     return blob, view, y.cpu().numpy()
 
 
+@pytest.mark.parametrize("checked", [True, False])
 @pytest.mark.parametrize("B", [1, 2, 3, 4, 5, 6, 7, 8])
 @pytest.mark.parametrize("shape", [(1, 128), (3, 384), (149, 640), (300, 1152), (77, 4096), (19, 14336)])
-def test_gemv_small_shapes_all_batches(s12, oracle, B, shape):
-    """Shapes that span several stages, a ragged row tail, partial 512-wide
-    column slots and (for B*K*2 > 96 KB) the multi-phase column split."""
+def test_gemv_small_shapes_all_batches(s12, oracle, B, shape, checked):
+    """Ragged 16-row groups, row groups split across many warps (stream-K
+    fix-up), x staged in shared memory or (B=8, K=14336) read from global
+    memory; with the error word (every tile checked) and without it."""
     r, c = shape
     w = wl.normal_with_outliers(r, c, 0.02, 0.002, r + c)
     x = wl.activations(B, c, B)
-    flag = new_flag()
-    blob, view, y = _gemv(s12, w, x, flag)
+    flag = new_flag() if checked else None
+    ws = torch.zeros(s12.s12_gemv_ws_bytes(s12.s12_open(s12.s12_encode(to_dev(w))), B), dtype=torch.uint8,
+                     device="cuda")
+    blob, view, y = _gemv(s12, w, x, flag, ws)
     yr, sr = oracle.gemv_f64(oracle.encode(w), x)
     assert_within_tolerance(y, yr, sr)
-    assert int(flag.item()) == 0
+    if checked:
+        assert int(flag.item()) == 0
+    # the arrival counters (the workspace's tail, one per 16-row group) are
+    # back at zero for the next call
+    n_cnt = -(-((view.rows + 15) // 16) * 4 // 256) * 256
+    assert int(ws[-n_cnt:].count_nonzero()) == 0
 
 
 def test_gemv_one_hot_is_exact(s12, oracle):
@@ -76,6 +85,25 @@ def test_gemv_escape_heavy(s12, oracle):
     yr, sr = oracle.gemv_f64(oracle.encode(w), x)
     assert_within_tolerance(y, yr, sr)
     assert int(flag.item()) == 0
+
+
+def test_gemv_workspace_reused_across_matrices(s12, oracle):
+    """One workspace serves a sequence of calls on different shapes (the
+    counters return to zero after every call), and a short one is refused."""
+    shapes = [(1024, 4096), (16, 14336), (4096, 1024), (33, 256), (1024, 4096)]
+    mats = [wl.student_t_scaled(r, c, i) for i, (r, c) in enumerate(shapes)]
+    views = [s12.s12_open(s12.s12_encode(to_dev(w))) for w in mats]
+    need = max(s12.s12_gemv_ws_bytes(v, 1) for v in views)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for i, (w, v) in enumerate(zip(mats, views)):
+        x = wl.activations(2, w.shape[1], i)
+        y = s12.s12_gemv(v, to_dev(x), ws=ws)
+        torch.cuda.synchronize()
+        yr, sr = oracle.matmul_f64(w, x)
+        assert_within_tolerance(y.cpu().numpy(), yr, sr)
+    small = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(s12.S12Error):
+        s12.s12_gemv(views[0], to_dev(wl.activations(1, 4096, 0)), ws=small)
 
 
 def test_gemv_deterministic(s12):
@@ -121,3 +149,52 @@ def test_bf16_baseline(s12, oracle, B, shape):
     torch.cuda.synchronize()
     yr, sr = oracle.matmul_f64(w, x)
     assert_within_tolerance(y.cpu().numpy(), yr, sr)
+
+
+@pytest.mark.parametrize("checked", [True, False])
+@pytest.mark.parametrize("B", [1, 3, 8])
+def test_gemv_multi_mixed_shapes(s12, oracle, B, checked):
+    """One grouped launch over matrices of different shapes (ragged row
+    groups, one-tile rows, long rows, escape-heavy rows) equals the oracle
+    for every member."""
+    shapes = [(77, 4096), (16, 14336), (300, 1152), (1, 128), (64, 2048), (33, 256)]
+    mats = [wl.normal_with_outliers(r, c, 0.02, 0.002, 100 + i) for i, (r, c) in enumerate(shapes)]
+    esc, _ = wl.escape_stress(0.10, 1, 64, 2048)
+    mats[4] = esc
+    xs = [wl.activations(B, c, 200 + i) for i, (_, c) in enumerate(shapes)]
+    views = [s12.s12_open(s12.s12_encode(to_dev(w))) for w in mats]
+    flag = new_flag() if checked else None
+    ys = s12.s12_gemv_multi(views, [to_dev(x) for x in xs], err_flag=flag)
+    torch.cuda.synchronize()
+    for w, x, y in zip(mats, xs, ys):
+        yr, sr = oracle.gemv_f64(oracle.encode(w), x)
+        assert_within_tolerance(y.cpu().numpy(), yr, sr)
+    if checked:
+        assert int(flag.item()) == 0
+
+
+def test_gemv_multi_llama_layer_matches_single_calls(s12):
+    """The grouped launch over a full 8B-style layer gives, per matrix, the
+    same y as separate s12_gemv calls up to the summation order (both are
+    checked against the oracle elsewhere), and is repeatable bit for bit."""
+    mats, xs = wl.llama8b_layer(0, 4)
+    names = list(wl.LLAMA8B_SHAPES)
+    views = [s12.s12_open(s12.s12_encode(to_dev(mats[n]))) for n in names]
+    xd = [to_dev(xs[n]) for n in names]
+    ws = torch.zeros(s12.s12_gemv_multi_ws_bytes(views, 4), dtype=torch.uint8, device="cuda")
+    a = s12.s12_gemv_multi(views, xd, ws=ws)
+    b = s12.s12_gemv_multi(views, xd, ws=ws)
+    singles = [s12.s12_gemv(v, x) for v, x in zip(views, xd)]
+    torch.cuda.synchronize()
+    for ya, yb, ys in zip(a, b, singles):
+        assert torch.equal(ya, yb)
+        scale = ys.abs().max().item()
+        assert torch.allclose(ya, ys, rtol=0, atol=1e-4 * scale)
+
+
+def test_gemv_multi_rejects_bad_groups(s12):
+    w = wl.student_t_scaled(64, 256, 0)
+    v = s12.s12_open(s12.s12_encode(to_dev(w)))
+    x = to_dev(wl.activations(1, 256, 0))
+    with pytest.raises(s12.S12Error):
+        s12.s12_gemv_multi([v] * 9, [x] * 9)
