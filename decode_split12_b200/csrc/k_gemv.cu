@@ -184,6 +184,23 @@ __device__ __forceinline__ Meta load_meta(const Problem &m_, Pos ps, int g) {
     return m;
 }
 
+// Metadata of the block after `prev` in the same row group (ps.j > 0): a
+// tile's first escape offset is the previous tile's end, so only the base
+// and the new end are read.
+__device__ __forceinline__ Meta load_meta_next(const Problem &m_, Pos ps, int g, const Meta &prev) {
+    const int rA = ps.grp * kRowsPerGroup + g, rB = rA + 8;
+    const size_t tA = static_cast<size_t>(min(rA, m_.R - 1)) * m_.T + ps.j;
+    const size_t tB = static_cast<size_t>(min(rB, m_.R - 1)) * m_.T + ps.j;
+    Meta m;
+    m.baseA = __ldg(m_.base + tA);
+    m.baseB = __ldg(m_.base + tB);
+    m.loA = prev.hiA;
+    m.loB = prev.hiB;
+    m.hiA = rA < m_.R ? __ldg(m_.esc_off + tA + 1) : m.loA;
+    m.hiB = rB < m_.R ? __ldg(m_.esc_off + tB + 1) : m.loB;
+    return m;
+}
+
 // The first escape value of a tile with escapes (0 otherwise), fetched ahead
 // of its use.
 __device__ __forceinline__ uint32_t first_escape(const Problem &m_, uint32_t lo, uint32_t hi) {
@@ -266,25 +283,24 @@ __device__ __noinline__ void finish_group(const Params &pr, float4 a4, Pos ps, l
 }
 
 // Escapes of one tile row for this lane (set up only for rows whose tile has
-// escapes): the escape-nibble masks of the lane's two chunks, the stream
-// index of each chunk's first escape, the end of the tile's escapes, and the
-// tile's first escape (index and prefetched value).
+// escapes): the stream index of the first escape of each of the lane's two
+// chunks, the end of the tile's escapes, and which chunks have any.
 struct EscRow {
-    uint2 m0, m1;
-    uint32_t s0, s1, limit, first, first_val;
+    uint32_t s0, s1, limit, has;  // has: bit h set if chunk h holds an escape
 };
 
 __device__ __forceinline__ uint32_t count2(uint2 m) { return __popc(m.x) + __popc(m.y); }
+
+__device__ __forceinline__ uint2 esc_mask(uint2 c) { return make_uint2(escape_nibbles(c.x), escape_nibbles(c.y)); }
 
 // Called by whole quads (the lanes of `quads`, a union of complete quads that
 // share a tile row).  Chunk order within a tile row: lane q = 0..3, half 0
 // then half 1 (chunk 2q + h covers columns 32q + 16h .. +15).  The tile's
 // code-15 count is checked against its esc_off span.
-__device__ __forceinline__ void prepare_row(uint4 c, uint32_t lo, uint32_t hi, uint32_t fv, uint64_t n_esc,
-                                            uint32_t *err, unsigned quads, int q, EscRow &e) {
-    e.m0 = make_uint2(escape_nibbles(c.x), escape_nibbles(c.y));
-    e.m1 = make_uint2(escape_nibbles(c.z), escape_nibbles(c.w));
-    const uint32_t n0 = count2(e.m0), n = n0 + count2(e.m1);
+__device__ __forceinline__ EscRow prepare_row(uint4 c, uint32_t lo, uint32_t hi, uint64_t n_esc, uint32_t *err,
+                                              unsigned quads, int q) {
+    const uint32_t n0 = count2(esc_mask(make_uint2(c.x, c.y))), n1 = count2(esc_mask(make_uint2(c.z, c.w)));
+    const uint32_t n = n0 + n1;
     uint32_t incl = n;
 #pragma unroll
     for (int d = 1; d < 4; d <<= 1) {
@@ -292,45 +308,55 @@ __device__ __forceinline__ void prepare_row(uint4 c, uint32_t lo, uint32_t hi, u
         if (q >= d) incl += v;
     }
     const uint32_t tot = __shfl_sync(quads, incl, 3, 4);
+    EscRow e;
     e.s0 = lo + incl - n;
     e.s1 = e.s0 + n0;
     e.limit = lo <= hi ? static_cast<uint32_t>(hi < n_esc ? hi : n_esc) : 0u;
-    e.first = lo;
-    e.first_val = fv;
+    e.has = (n0 ? 1u : 0u) | (n1 ? 2u : 0u);
     if (q == 0 && tot != hi - lo) raise_flag(err, S12_FLAG_ESC_COUNT);
+    return e;
 }
 
-// A chunk with escapes: decode it again with the escape nibbles cleared (so
-// base + code never carries out of a byte, even for base 241), then put the
-// exact value of each escaped weight in place, reading the stream from
-// index `idx`; reads at or past the tile's end are skipped and flagged.
-__device__ __forceinline__ void fix_chunk(uint32_t (&w)[8], uint4 raw, uint2 code, uint32_t base, uint2 m,
-                                          uint32_t idx, const EscRow &e, const uint16_t *__restrict__ esc,
-                                          uint32_t *err) {
-    decode16(raw, make_uint2(clear_escapes(code.x, m.x), clear_escapes(code.y, m.y)), base * 0x01010101u, w);
-    uint32_t m0 = m.x, m1 = m.y;
-    while (m0 | m1) {
-        int j;
-        if (m0) {
-            j = (__ffs(m0) - 1) >> 2;
-            m0 &= m0 - 1;
-        } else {
-            j = 8 + ((__ffs(m1) - 1) >> 2);
-            m1 &= m1 - 1;
-        }
+// A chunk with escapes: put the exact value of each escaped weight in place,
+// reading the stream from index `idx`; reads at or past the tile's end are
+// skipped and flagged.  The decoded words go through the lane's 32-byte
+// shared-memory scratch `sc`, so a weight is replaced by one 16-bit store
+// at its position.  With base <= 240, base + 15 stays inside its byte and
+// the other weights of the chunk are already right; a base of 241 could
+// carry into the next byte, so such chunks are decoded again with the
+// escape nibbles cleared first.
+__device__ __forceinline__ void fix_chunk(uint32_t (&w)[8], uint4 raw, uint2 code, uint32_t base, uint32_t idx,
+                                          uint32_t limit, uint32_t first, uint32_t first_val,
+                                          const uint16_t *__restrict__ esc, uint32_t *err, uint32_t sc) {
+    const uint2 m = esc_mask(code);
+    if (base > static_cast<uint32_t>(kMaxBase - 1))
+        decode16(raw, make_uint2(clear_escapes(code.x, m.x), clear_escapes(code.y, m.y)), base * 0x01010101u, w);
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sc), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
+                 : "memory");
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sc + 16), "r"(w[4]), "r"(w[5]), "r"(w[6]),
+                 "r"(w[7])
+                 : "memory");
+    // nibble j of the chunk is 15  <=>  bit 4j+3 of the 64-bit mask
+    uint64_t mm = (static_cast<uint64_t>(m.y) << 32) | m.x;
+    while (mm) {
+        const int j = (__ffsll(static_cast<long long>(mm)) - 1) >> 2;
+        mm &= mm - 1;
         uint32_t v = 0;
-        if (idx < e.limit)
-            v = idx == e.first ? e.first_val : __ldg(esc + idx);
+        if (idx < limit)
+            v = idx == first ? first_val : __ldg(esc + idx);
         else
             raise_flag(err, S12_FLAG_ESC_RANGE);
         ++idx;
-        const int r = j >> 1;
-        const uint32_t keep = (j & 1) ? 0x0000FFFFu : 0xFFFF0000u;
-        const uint32_t put = (j & 1) ? (v << 16) : v;
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            if (i == r) w[i] = (w[i] & keep) | put;
+        asm volatile("st.shared.u16 [%0], %1;" ::"r"(sc + 2u * j), "h"(static_cast<uint16_t>(v)) : "memory");
     }
+    uint4 a, b;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w) : "r"(sc)
+                 : "memory");
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+                 : "r"(sc + 16)
+                 : "memory");
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+    w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
 }
 
 __device__ __forceinline__ float4 sum_halves(const float (&acc)[2][4]) {
@@ -380,6 +406,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_tma_kernel(const __grid_c
     const int S = pr.stages;
     const uint32_t bars = sb + static_cast<uint32_t>(warp) * kMaxStages * 8u;
     const uint32_t ring = sb + kRingOff + static_cast<uint32_t>(warp * S) * kStageBytes;
+    const uint32_t scr = sb + kRingOff + static_cast<uint32_t>(kWarps * S) * kStageBytes + threadIdx.x * 32u;
     if (threadIdx.x == 0) grid_launch_dependents();
 
     // The weights are never written by other kernels: start the copies
@@ -406,7 +433,6 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_tma_kernel(const __grid_c
     const uint32_t oCA = kRawBytes + g * 64 + 16 * q, oCB = oCA + 8 * 64;
 
     Pos pc = p0;  // block being computed
-    Pos pn = p0;  // block whose first escapes are fetched (one ahead)
     Pos pm = p0;  // block whose metadata is loaded (two ahead)
     Meta m0 = load_meta(pr.prob[pm.p], pm, g), m1 = m0;
     advance(pm, pr);
@@ -423,11 +449,12 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_tma_kernel(const __grid_c
         Meta m2 = m1;
         if (i + 2 < nb) {
             advance(pm, pr);
-            m2 = load_meta(pr.prob[pm.p], pm, g);
+            m2 = pm.j > 0 ? load_meta_next(pr.prob[pm.p], pm, g, m1) : load_meta(pr.prob[pm.p], pm, g);
         }
         uint32_t nfvA = 0, nfvB = 0;
         if (i + 1 < nb) {
-            advance(pn, pr);  // now the position of block i + 1
+            Pos pn = pc;
+            advance(pn, pr);  // the position of block i + 1
             const Problem &mn = pr.prob[pn.p];
             nfvA = first_escape(mn, m1.loA, m1.hiA);
             nfvB = first_escape(mn, m1.loB, m1.hiB);
@@ -438,7 +465,6 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_tma_kernel(const __grid_c
             for (int k = 0; k < 4; ++k) acc[0][k] = acc[1][k] = 0.f;
             cur = pc;
         }
-        const Problem &mp = pr.prob[pc.p];
         const uint32_t bar = bars + 8u * s;
         if (!__all_sync(0xFFFFFFFFu, mbar_wait_s(bar, parity))) {
             raise_flag(pr.err, S12_FLAG_TIMEOUT);
@@ -446,40 +472,44 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_tma_kernel(const __grid_c
             break;
         }
         const uint32_t st = ring + s * kStageBytes;
+        bool esc = (m0.loA != m0.hiA) || (m0.loB != m0.hiB);
+        if (CHECK) {
+            const uint4 cA = lds128(st + oCA), cB = lds128(st + oCB);
+            esc = esc || (escape_nibbles(cA.x) | escape_nibbles(cA.y) | escape_nibbles(cA.z) | escape_nibbles(cA.w) |
+                          escape_nibbles(cB.x) | escape_nibbles(cB.y) | escape_nibbles(cB.z) | escape_nibbles(cB.w)) != 0;
+            if (m0.baseA > static_cast<uint32_t>(kMaxBase) || m0.baseB > static_cast<uint32_t>(kMaxBase))
+                raise_flag(pr.err, S12_FLAG_BASE);
+        }
+        const Problem &mp = pr.prob[pc.p];
+        const uint16_t *xl = mp.x + static_cast<size_t>(gx) * mp.K + 32 * q;
         const uint4 rA0 = lds128(st + oA0), rA1 = lds128(st + oA1), rB0 = lds128(st + oB0), rB1 = lds128(st + oB1);
         const uint4 cA = lds128(st + oCA), cB = lds128(st + oCB);
         // the stage is in registers: hand it back to the copy engine
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
         if (lane == 0 && i + S < nb) copy_block(pr, pi, st, bar, pol);
-        if (i + S < nb) advance(pi, pr);
-
-        bool escA = m0.loA != m0.hiA, escB = m0.loB != m0.hiB;
-        if (CHECK) {
-            escA = escA || (escape_nibbles(cA.x) | escape_nibbles(cA.y) | escape_nibbles(cA.z) | escape_nibbles(cA.w));
-            escB = escB || (escape_nibbles(cB.x) | escape_nibbles(cB.y) | escape_nibbles(cB.z) | escape_nibbles(cB.w));
-            if (m0.baseA > static_cast<uint32_t>(kMaxBase) || m0.baseB > static_cast<uint32_t>(kMaxBase))
-                raise_flag(pr.err, S12_FLAG_BASE);
-        }
-        const unsigned qA = __ballot_sync(0xFFFFFFFFu, escA), qB = __ballot_sync(0xFFFFFFFFu, escB);
-        const bool any = (qA | qB) != 0;
-        EscRow eA, eB;
+        const bool any = __any_sync(0xFFFFFFFFu, esc);
+        EscRow eA = {0, 0, 0, 0}, eB = {0, 0, 0, 0};
         if (any) {
-            if (escA) prepare_row(cA, m0.loA, m0.hiA, fvA, mp.n_esc, pr.err, qA, q, eA);
-            if (escB) prepare_row(cB, m0.loB, m0.hiB, fvB, mp.n_esc, pr.err, qB, q, eB);
+            const bool escA = m0.loA != m0.hiA || (escape_nibbles(cA.x) | escape_nibbles(cA.y) |
+                                                   escape_nibbles(cA.z) | escape_nibbles(cA.w)) != 0;
+            const bool escB = m0.loB != m0.hiB || (escape_nibbles(cB.x) | escape_nibbles(cB.y) |
+                                                   escape_nibbles(cB.z) | escape_nibbles(cB.w)) != 0;
+            const unsigned qA = __ballot_sync(0xFFFFFFFFu, escA), qB = __ballot_sync(0xFFFFFFFFu, escB);
+            if (escA) eA = prepare_row(cA, m0.loA, m0.hiA, mp.n_esc, pr.err, qA, q);
+            if (escB) eB = prepare_row(cB, m0.loB, m0.hiB, mp.n_esc, pr.err, qB, q);
         }
         const uint32_t B4A = m0.baseA * 0x01010101u, B4B = m0.baseB * 0x01010101u;
-        const uint16_t *xl = mp.x + static_cast<size_t>(gx) * mp.K + 32 * q;
         uint32_t xw[8], wa[8], wb[8];
         // half 0
         load_x(xw, xl, pc.j, 0);
         decode16(rA0, make_uint2(cA.x, cA.y), B4A, wa);
         decode16(rB0, make_uint2(cB.x, cB.y), B4B, wb);
         if (any) {
-            if (escA && (eA.m0.x | eA.m0.y))
-                fix_chunk(wa, rA0, make_uint2(cA.x, cA.y), m0.baseA, eA.m0, eA.s0, eA, mp.esc, pr.err);
-            if (escB && (eB.m0.x | eB.m0.y))
-                fix_chunk(wb, rB0, make_uint2(cB.x, cB.y), m0.baseB, eB.m0, eB.s0, eB, mp.esc, pr.err);
+            if (eA.has & 1u)
+                fix_chunk(wa, rA0, make_uint2(cA.x, cA.y), m0.baseA, eA.s0, eA.limit, m0.loA, fvA, mp.esc, pr.err, scr);
+            if (eB.has & 1u)
+                fix_chunk(wb, rB0, make_uint2(cB.x, cB.y), m0.baseB, eB.s0, eB.limit, m0.loB, fvB, mp.esc, pr.err, scr);
         }
         half_mma(acc[0], wa, wb, xw);
         // half 1
@@ -487,12 +517,13 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_tma_kernel(const __grid_c
         decode16(rA1, make_uint2(cA.z, cA.w), B4A, wa);
         decode16(rB1, make_uint2(cB.z, cB.w), B4B, wb);
         if (any) {
-            if (escA && (eA.m1.x | eA.m1.y))
-                fix_chunk(wa, rA1, make_uint2(cA.z, cA.w), m0.baseA, eA.m1, eA.s1, eA, mp.esc, pr.err);
-            if (escB && (eB.m1.x | eB.m1.y))
-                fix_chunk(wb, rB1, make_uint2(cB.z, cB.w), m0.baseB, eB.m1, eB.s1, eB, mp.esc, pr.err);
+            if (eA.has & 2u)
+                fix_chunk(wa, rA1, make_uint2(cA.z, cA.w), m0.baseA, eA.s1, eA.limit, m0.loA, fvA, mp.esc, pr.err, scr);
+            if (eB.has & 2u)
+                fix_chunk(wb, rB1, make_uint2(cB.z, cB.w), m0.baseB, eB.s1, eB.limit, m0.loB, fvB, mp.esc, pr.err, scr);
         }
         half_mma(acc[1], wa, wb, xw);
+        if (i + S < nb) advance(pi, pr);
 
         advance(pc, pr);
         m0 = m1;
@@ -583,8 +614,9 @@ int run(const s12_view *views, int count, const uint16_t *const *x, int B, float
     pr.B = B;
     pr.n_units = pl.n_units;
     pr.stages = gemv::kMaxStages;
-    // 1 KB alignment slack, barriers, then the warps' rings
-    const uint32_t smem = 1024 + gemv::kRingOff + gemv::kWarps * pr.stages * gemv::kStageBytes;
+    // 1 KB alignment slack, barriers, the warps' rings, 32 bytes of escape
+    // scratch per lane
+    const uint32_t smem = 1024 + gemv::kRingOff + gemv::kWarps * pr.stages * gemv::kStageBytes + gemv::kWarps * 32 * 32;
     if (smem > kSmemLimit) return S12_ERR_CUDA;
     auto kern = gemv::gemv_tma_kernel<CHECK>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
