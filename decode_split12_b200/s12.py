@@ -34,7 +34,8 @@ S12_FLAG_TIMEOUT = 8
 
 EXPORTED = (
     "s12_error_string", "s12_device_check", "s12_container_bytes", "s12_encode_ws_bytes", "s12_encode",
-    "s12_open", "s12_decode", "s12_gemv_ws_bytes", "s12_gemv", "s12_gemv_multi_ws_bytes", "s12_gemv_multi", "s12_gemm_ws_bytes", "s12_gemm_skinny", "s12_stats_ws_bytes",
+    "s12_open", "s12_decode", "s12_gemv_ws_bytes", "s12_gemv", "s12_gemv_multi_ws_bytes", "s12_gemv_multi",
+    "s12_gemv_noalloc", "s12_gemm_ws_bytes", "s12_gemm_skinny", "s12_stats_ws_bytes",
     "s12_stats", "s12_bf16_gemv",
 )
 
@@ -98,6 +99,8 @@ def _lib() -> C.CDLL:
         lib.s12_gemv_multi.argtypes = [C.POINTER(View), C.c_int, C.POINTER(_P), C.c_int, C.POINTER(_P), _P, _SZ, _P,
                                        _P]
         lib.s12_gemv_multi.restype = C.c_int
+        lib.s12_gemv_noalloc.argtypes = [C.POINTER(View), _P, C.c_int, _P, _P, _P]
+        lib.s12_gemv_noalloc.restype = C.c_int
         lib.s12_gemv.restype = C.c_int
         lib.s12_gemm_ws_bytes.argtypes = [C.POINTER(View), C.c_int]
         lib.s12_gemm_ws_bytes.restype = _SZ
@@ -265,6 +268,18 @@ def s12_gemv_multi(views, xs, ys=None, ws: torch.Tensor | None = None, err_flag:
     _check(_lib().s12_gemv_multi(arr, len(views), xp, B, yp, _dptr(ws), ws.numel(), _dptr(err_flag),
                                  _stream(stream)), "s12_gemv_multi")
     return ys
+
+
+def s12_gemv_noalloc(view: View, x: torch.Tensor, y: torch.Tensor | None = None,
+                     err_flag: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """s12_gemv without a caller workspace (the library's static one)."""
+    x = _u16(x)
+    B = x.shape[0] if x.dim() == 2 else 1
+    if y is None:
+        y = torch.empty((B, view.rows), dtype=torch.float32, device=x.device)
+    _check(_lib().s12_gemv_noalloc(C.byref(view), _dptr(x), B, _dptr(y), _dptr(err_flag), _stream(stream)),
+           "s12_gemv_noalloc")
+    return y
 
 
 def s12_gemm_ws_bytes(view: View, M: int) -> int:

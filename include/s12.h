@@ -212,6 +212,28 @@ size_t s12_gemv_multi_ws_bytes(const s12_view *views, int count, int B);
 int s12_gemv_multi(const s12_view *views, int count, const uint16_t *const *x, int B, float *const *y,
                    void *ws, size_t ws_bytes, uint32_t *err_flag, void *stream);
 
+/* s12_gemv for callers that cannot allocate device memory (no counterpart
+ * in the pages: it exists for integration, not for the method).  Examples are
+ * a plugin whose host engine owns all device memory through its own
+ * allocator, code under a fixed memory budget, or a path where cudaMalloc's
+ * implicit synchronisation is not allowed.  Same arguments and result as
+ * s12_gemv, minus the workspace.  Instead, the call uses a 2.75 MiB workspace
+ * that is a static array inside the library, reserved on every device that
+ * loads the library and held until the process exits.
+ *   - Limits: containers of at most 2^20 rows, devices of at most 160 SMs;
+ *     beyond them S12_ERR_CAPACITY, before any device work.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and caches it; make that first call outside any
+ *     stream capture.
+ *   - Each call first clears its arrival counters with an asynchronous
+ *     memset on `stream`, then runs the s12_gemv kernel.  It allocates and
+ *     frees nothing.
+ *   - All calls share one array, which keeps the last call's contents.
+ *     Calls that can overlap on the GPU (different streams without ordering)
+ *     race on it and give wrong results; serialise them or use s12_gemv. */
+int s12_gemv_noalloc(const s12_view *v, const uint16_t *x, int B, float *y, uint32_t *err_flag,
+                     void *stream);
+
 /* ---- fused decode-skinny-GEMM on tcgen05 tensor cores ---- */
 
 /* Workspace bytes s12_gemm_skinny needs for this container and M. */
