@@ -17,6 +17,10 @@ cudaError_t device_sms(int *sms);
 // the 128-byte swizzle), out-of-bounds bytes read as 0.
 int make_tmap_u8_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t rows, uint64_t row_stride,
                     uint32_t box_inner, uint32_t box_rows, bool swizzle128);
+// The same for a row-major 2-D array of BF16 values (`inner` and the box's
+// inner extent counted in elements, `row_stride` in bytes).
+int make_tmap_bf16_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t rows, uint64_t row_stride,
+                      uint32_t box_inner, uint32_t box_rows, bool swizzle128);
 
 int launch_decode(const s12_view *v, uint16_t *out, uint32_t *err, cudaStream_t stream);
 size_t gemv_ws_bytes(const s12_view *views, int count);
