@@ -379,6 +379,13 @@ def cpu_baseline_llama(target_s: float = 12.0):
                       f"{weights} weights in {secs:.1f} s on 1 of {os.cpu_count()} host cores"}
 
 
+def llama_config(batch: int) -> dict:
+    """The workload both arms (library and oracle) report."""
+    return {"workload": f"llama8b-layer decode GEMV, B={batch}: q,o 4096x4096; k,v 1024x4096; "
+                        f"gate,up 14336x4096; down 4096x14336 (Student-t(5)/sqrt(in), Split12)",
+            "batch": batch}
+
+
 def run_llama8b(args, world, rank):
     import torch
     hbm, _, _, peak_kind = load_peaks()
@@ -432,6 +439,10 @@ def run_llama8b(args, world, rank):
                        "hbm_frac": round(2 * layer.weights / sb / 1e9 / hbm, 4)}
         del gb
     e2e_t, h2d, d2h, ge = e2e_llama(layer, max(20, args.steps // 2), args.warmup, world)
+    if not args.no_gemm:
+        del layer.w_dev
+        torch.cuda.empty_cache()
+        extra["gemm_70b_mlp_tcgen05"] = gemm_extras(world)
     del ge
     traffic = load_traffic("gemv_tma_kernel", f"llama8b_b{args.batch}")
     out = {
@@ -448,9 +459,7 @@ def run_llama8b(args, world, rank):
         "dtype": "f32",
         "data": "synthetic",
         "config": {
-            "workload": f"llama8b-layer decode GEMV, B={args.batch}: q,o 4096x4096; k,v 1024x4096; "
-                        f"gate,up 14336x4096; down 4096x14336 (Student-t(5)/sqrt(in), Split12 resident in HBM)",
-            "batch": args.batch,
+            **llama_config(args.batch),
             "weights_per_step": layer.weights,
             "compressed_bytes_per_step": layer.compressed,
             "algorithmic_bytes_per_step": layer.read_bytes,
@@ -478,6 +487,51 @@ def run_llama8b(args, world, rank):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline_llama()
+    return out
+
+
+def gemm_extras(world, steps: int = 40):
+    """The 70B-style MLP decode-phase skinny GEMM: W 28672x8192 and
+    8192x28672 (N(0, 1/sqrt(in)) with 0.05 % outliers x U(10, 100)), X bf16
+    N(0, 1) at M = 16..256, on the tcgen05 fused decode-GEMM, next to cuBLAS
+    (torch.matmul) on the uncompressed BF16 weights.  Each container (361 MB)
+    is larger than L2, so back-to-back calls stream it from HBM."""
+    import torch
+
+    from decode_split12_b200 import s12
+    hbm, tf_burst, tf_sust, _ = load_peaks()
+    out = {}
+    for name in wl.MLP70B_SHAPES:
+        w = wl.mlp70b(name, 0)
+        wd = dev16(w)
+        del w
+        blob = s12.s12_encode(wd)
+        view = s12.s12_open(blob)
+        n, k = int(view.rows), int(view.cols)
+        cbytes = int(view.container_bytes)
+        res = {}
+        for m in (16, 32, 64, 128, 256):
+            x = dev16(wl.activations(m, k, m))
+            y = torch.empty((m, n), dtype=torch.float32, device="cuda")
+            ws = torch.zeros(s12.s12_gemm_ws_bytes(view, m), dtype=torch.uint8, device="cuda")
+            g = capture(lambda: s12.s12_gemm_skinny(view, x, y, ws=ws))
+            for _ in range(3):
+                g.replay()
+            t = time_graph(g, steps, world) / steps
+            gb = capture(lambda: torch.matmul(x.view(torch.bfloat16), wd.view(torch.bfloat16).t()))
+            for _ in range(3):
+                gb.replay()
+            tb = time_graph(gb, steps, world) / steps
+            alg = n * k * 3 // 2 + (n * k // 128) * 5 + 2 * int(view.n_esc) + m * k * 2 + m * n * 4
+            flops = 2.0 * m * n * k
+            res[f"M{m}"] = {"us": round(t * 1e6, 2), "hbm_GBs": round(alg / t / 1e9, 1),
+                            "hbm_frac": round(alg / t / 1e9 / hbm, 4), "TFLOPs": round(flops / t / 1e12, 1),
+                            "tensor_frac_sustained": round(flops / t / 1e12 / tf_sust, 4),
+                            "cublas_bf16_us": round(tb * 1e6, 2)}
+            del g, gb
+        out[f"{name}_{n}x{k}"] = {"container_bytes": cbytes, **res}
+        del wd, blob
+        torch.cuda.empty_cache()
     return out
 
 
@@ -517,8 +571,7 @@ def run_reference(args, world, rank):
     return {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(t_step * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"llama8b-layer decode GEMV, B={args.batch} (oracle on a 1% row sample)",
-                       "batch": args.batch},
+            "config": llama_config(args.batch),
             "impl": "reference", "cpu_baseline": cb,
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
@@ -602,6 +655,7 @@ def main(argv=None):
     ap.add_argument("--workload", choices=["llama8b", "single"], default="llama8b")
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-gemm", action="store_true", help="skip the skinny-GEMM extras")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3

@@ -11,7 +11,7 @@
 // decompression-GEMM; "GPU 友善 12 位無損 BF16 壓縮格式", key points: the
 // integer-ADD decode feeding tensor-core kernels).
 //
-// One CTA per SM, ten warps with fixed roles:
+// One CTA per SM, eighteen warps with fixed roles:
 //   warp 0      TMA producer: per 64-column chunk of a 128-row tile, the raw
 //               plane (128 x 64 bytes), the code plane (128 x 32 bytes) and
 //               the X chunk (M x 64 bf16, 128-byte swizzle) into a ring of
@@ -21,7 +21,7 @@
 //               decoded W chunk in shared memory, B = the X chunk, FP32
 //               accumulators in TMEM (128 lanes x M columns), and releases
 //               stages and A buffers with tcgen05.commit.
-//   warps 2..9  decode: each thread owns 16 weights of two rows per chunk,
+//   warps 2..17 decode: each thread owns 16 weights of one row per chunk,
 //               rebuilds the exact BF16 values (byte-wise base + code ADD,
 //               escapes patched from the escape stream) and stores them in
 //               the canonical K-major 128-byte-swizzled layout the tensor
@@ -47,12 +47,12 @@ namespace gemm {
 
 constexpr int kRows = 128;         // W rows per tile (UMMA M)
 constexpr int kChunk = 64;         // K columns per chunk (one 128-byte swizzle atom of bf16)
-constexpr int kDecodeWarps = 8;
+constexpr int kDecodeWarps = 16;
 constexpr int kThreads = 32 * (2 + kDecodeWarps);
 constexpr uint32_t kRawBytes = kRows * kChunk;       // 8 KB
 constexpr uint32_t kCodeBytes = kRows * kChunk / 2;  // 4 KB
 constexpr uint32_t kABytes = kRows * kChunk * 2;     // 16 KB decoded chunk
-constexpr int kABufs = 2;
+constexpr int kABufs = 3;
 constexpr int kMaxStages = 6;
 
 struct __align__(64) Params {
@@ -96,7 +96,7 @@ __device__ __forceinline__ void bar_expect_tx(uint32_t bar, uint32_t bytes) {
 __device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity))
+    while (!mbar_try_wait_hint(bar, parity, 1000u))  // the thread may sleep up to 1 us per try
         if (clock64() - t0 > kWaitCycles) return false;
     return true;
 }
@@ -153,6 +153,14 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
 __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&v)[8]) {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
                  : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+                 : "r"(taddr)
+                 : "memory");
+}
+
+// 32 TMEM lanes x 4 consecutive 32-bit columns into 4 registers per thread.
+__device__ __forceinline__ void tmem_ld4(uint32_t taddr, uint32_t (&v)[4]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
                  : "r"(taddr)
                  : "memory");
 }
@@ -239,16 +247,44 @@ __device__ __forceinline__ Layout layout(uint32_t sb, const Params &p) {
 // Decode one 16-weight piece (row r of the tile, columns 16*q4 .. +15 of
 // the chunk) from the stage into the A buffer, patching escapes.  Called by
 // whole quads (the four lanes of a quad share the row).
+// Per-tile metadata of one row: base and escape offsets.
+struct RowMeta {
+    uint32_t base, lo, hi;
+    uint32_t fv0, fv1;  // the tile row's first two escape values (fetched one unit ahead)
+};
+
+__device__ __forceinline__ void fetch_escapes(const Params &p, RowMeta &m) {
+    m.fv0 = m.fv1 = 0;
+    if (m.lo < m.hi && m.lo < p.n_esc) m.fv0 = __ldg(p.esc + m.lo);
+    if (m.lo + 1 < m.hi && m.lo + 1 < p.n_esc) m.fv1 = __ldg(p.esc + m.lo + 1);
+}
+
+// Rows past the end (zeros from the copy engine) read the last row's
+// metadata but report no escapes.
+__device__ __forceinline__ RowMeta load_row_meta(const Params &p, long long unit, int r) {
+    const int tile = static_cast<int>(unit / p.n_chunks), j = static_cast<int>(unit % p.n_chunks) >> 1;
+    const int n = tile * kRows + r;
+    const size_t t = static_cast<size_t>(min(n, p.N - 1)) * p.T + j;
+    RowMeta m;
+    m.base = __ldg(p.base + t);
+    m.lo = __ldg(p.esc_off + t);
+    m.hi = __ldg(p.esc_off + t + 1);
+    if (n >= p.N) m.hi = m.lo;
+    m.fv0 = m.fv1 = 0;
+    return m;
+}
+
+// `carry` holds, after a first-half chunk of a tile row with escapes, that
+// half's escape count for the row (all four lanes of the quad); the
+// second-half chunk that follows uses it instead of re-reading the codes.
 template <bool CHECK>
 __device__ __forceinline__ void decode_piece(const Params &p, uint32_t st_raw, uint32_t st_code, uint32_t abuf,
-                                             int tile, int chunk, int r, int q4, unsigned full_mask) {
+                                             int tile, int chunk, int r, int q4, unsigned full_mask,
+                                             const RowMeta &rm, uint32_t &carry, bool carry_ok) {
     const int n = tile * kRows + r;
     const int j = chunk >> 1, h = chunk & 1;
     const int nc = min(n, p.N - 1);
-    const size_t t = static_cast<size_t>(nc) * p.T + j;
-    const uint32_t base = __ldg(p.base + t);
-    uint32_t lo = __ldg(p.esc_off + t), hi = __ldg(p.esc_off + t + 1);
-    if (n >= p.N) hi = lo;  // rows past the end (zeros from the copy engine) have no escapes
+    const uint32_t base = rm.base, lo = rm.lo, hi = rm.hi;
     const uint4 raw = lds128(st_raw + r * 64 + q4 * 16);
     uint2 code = lds64(st_code + r * 32 + q4 * 8);
     const uint32_t rowa = abuf + static_cast<uint32_t>(r) * 128u, sw = static_cast<uint32_t>(r & 7);
@@ -272,7 +308,9 @@ __device__ __forceinline__ void decode_piece(const Params &p, uint32_t st_raw, u
             if (q4 >= d) incl += v;
         }
         uint32_t before = 0;  // escapes of this tile row in the first half (columns 0..63)
-        if (h == 1) {
+        if (h == 1 && carry_ok) {
+            before = carry;
+        } else if (h == 1) {
             const uint2 c0 = __ldg(reinterpret_cast<const uint2 *>(p.code + static_cast<size_t>(nc) * (p.K / 2) +
                                                                    static_cast<size_t>(j) * 64 + q4 * 8));
             uint32_t n0 = __popc(escape_nibbles(c0.x)) + __popc(escape_nibbles(c0.y));
@@ -281,6 +319,7 @@ __device__ __forceinline__ void decode_piece(const Params &p, uint32_t st_raw, u
             before = n0;
         }
         const uint32_t total_half = __shfl_sync(quads, incl, 3, 4);
+        if (h == 0) carry = total_half;
         if (h == 1 && q4 == 0 && before + total_half != hi - lo) raise_flag(p.err, S12_FLAG_ESC_COUNT);
         if (h == 0 && q4 == 0 && total_half > hi - lo) raise_flag(p.err, S12_FLAG_ESC_COUNT);
         rank = lo + before + incl - cnt;
@@ -298,7 +337,8 @@ __device__ __forceinline__ void decode_piece(const Params &p, uint32_t st_raw, u
             mm &= mm - 1;
             uint16_t v = 0;
             if (idx < limit)
-                v = __ldg(p.esc + idx);
+                v = idx == lo ? static_cast<uint16_t>(rm.fv0)
+                              : (idx == lo + 1 ? static_cast<uint16_t>(rm.fv1) : __ldg(p.esc + idx));
             else
                 raise_flag(p.err, S12_FLAG_ESC_RANGE);
             ++idx;
@@ -316,26 +356,26 @@ namespace gemm {
 
 // Epilogue for tile `tile` (the accumulators are final for this CTA's part
 // of it): store Y directly, or hand the partial to the stream-K fix-up.
-// Run by the 256 decode threads (warps 2..9); ew = warp - 2.
+// Run by the 512 decode threads (warps 2..17); ew = warp - 2.
 __device__ __forceinline__ void epilogue(const Params &p, uint32_t tmem, const Layout &L, int tile, long long u0,
                                          long long u1, int ew, int lane) {
     const int warp = ew + 2;
     const int quad = warp & 3;                 // TMEM lanes 32*quad .. +31 are this warp's
     const int row = quad * 32 + lane;          // row within the tile
     const int n = tile * kRows + row;
-    const int half_cols = p.Mp / 2, c_begin = (ew >> 2) * half_cols;
+    const int part_cols = p.Mp / 4, c_begin = (ew >> 2) * part_cols;  // four warps share a lane quadrant
     const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const long long t0 = static_cast<long long>(tile) * p.n_chunks, t1 = t0 + p.n_chunks;
     const bool whole = t0 >= u0 && t1 <= u1;
     const int cta = blockIdx.x;
     const int slot = (tile == static_cast<int>(u0 / p.n_chunks)) ? 0 : 1;
     float *mine = p.part + (static_cast<size_t>(cta) * 2 + slot) * static_cast<size_t>(p.Mp) * kRows;
-    for (int c = c_begin; c < c_begin + half_cols; c += 8) {
-        uint32_t v[8];
-        tmem_ld8(taddr + static_cast<uint32_t>(c), v);
+    for (int c = c_begin; c < c_begin + part_cols; c += 4) {
+        uint32_t v[4];
+        tmem_ld4(taddr + static_cast<uint32_t>(c), v);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 4; ++i) {
             const int m = c + i;
             if (whole) {
                 if (m < p.M && n < p.N) p.y[static_cast<size_t>(m) * p.N + n] = __uint_as_float(v[i]);
@@ -364,7 +404,6 @@ __device__ __forceinline__ void epilogue(const Params &p, uint32_t tmem, const L
     asm volatile("ld.shared.u32 %0, [%1];" : "=r"(last) : "r"(L.xchg) : "memory");
     if (!last) return;
     __threadfence();
-    // 256 threads: thread (ew, lane) sums rows row2 = ew*16 + (lane>>1) ... for all m, by columns
     for (int idx = ew * 32 + lane; idx < p.Mp * kRows; idx += 32 * kDecodeWarps) {
         const int m = idx / kRows, r = idx - m * kRows;
         float s = 0.f;
@@ -489,12 +528,23 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         // ---- decode warps (and the epilogue)
         const int ew = warp - 2;
         const int t = ew * 32 + lane;
-        const int q4 = t & 3, rp = t >> 2;  // rows rp and rp + 64 of each chunk
+        const int q4 = t & 3, r = t >> 2;  // row r of each chunk, columns 16*q4 .. +15
         int s = 0, a = 0;
         uint32_t round = 0, around = 0, tiles = 0;
+        // the row metadata of the next two units is in flight while a unit is decoded
+        RowMeta m0 = {0, 0, 0, 0, 0}, m1 = {0, 0, 0, 0, 0};
+        if (u0 < u1) {
+            m0 = load_row_meta(p, u0, r);
+            fetch_escapes(p, m0);
+        }
+        if (u0 + 1 < u1) m1 = load_row_meta(p, u0 + 1, r);
+        uint32_t carry = 0;
         for (long long u = u0; u < u1; ++u) {
             const int tile = static_cast<int>(u / p.n_chunks), chunk = static_cast<int>(u % p.n_chunks);
             const bool last = (u + 1 == u1) || chunk == p.n_chunks - 1;
+            RowMeta m2 = m1;
+            if (u + 2 < u1) m2 = load_row_meta(p, u + 2, r);
+            if (u + 1 < u1) fetch_escapes(p, m1);  // m1's offsets arrived during the previous unit
             const bool w = bar_wait(L.full + 8 * s, round & 1u) && bar_wait(L.a_empty + 8 * a, (around & 1u) ^ 1u);
             if (!__all_sync(0xFFFFFFFFu, w)) {
                 raise_flag(p.err, S12_FLAG_TIMEOUT);
@@ -502,9 +552,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             }
             const uint32_t st = L.stages + static_cast<uint32_t>(s) * p.stage_bytes;
             const uint32_t aa = L.abuf + static_cast<uint32_t>(a) * kABytes;
-            decode_piece<CHECK>(p, st + p.x_bytes, st + p.x_bytes + kRawBytes, aa, tile, chunk, rp, q4, 0xFFFFFFFFu);
-            decode_piece<CHECK>(p, st + p.x_bytes, st + p.x_bytes + kRawBytes, aa, tile, chunk, rp + 64, q4,
-                                0xFFFFFFFFu);
+            decode_piece<CHECK>(p, st + p.x_bytes, st + p.x_bytes + kRawBytes, aa, tile, chunk, r, q4, 0xFFFFFFFFu, m0,
+                                carry, u > u0);
+            m0 = m1;
+            m1 = m2;
             // generic-proxy stores must be visible to the tensor core
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();

@@ -488,41 +488,46 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_tma_kernel(const __grid_c
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
         if (lane == 0 && i + S < nb) copy_block(pr, pi, st, bar, pol);
-        const bool any = __any_sync(0xFFFFFFFFu, esc);
-        EscRow eA = {0, 0, 0, 0}, eB = {0, 0, 0, 0};
-        if (any) {
+        const uint32_t B4A = m0.baseA * 0x01010101u, B4B = m0.baseB * 0x01010101u;
+        uint32_t xw[8], wa[8], wb[8];
+        if (!__any_sync(0xFFFFFFFFu, esc)) {
+            // no escapes in the block: straight decode and products
+            load_x(xw, xl, pc.j, 0);
+            decode16(rA0, make_uint2(cA.x, cA.y), B4A, wa);
+            decode16(rB0, make_uint2(cB.x, cB.y), B4B, wb);
+            half_mma(acc[0], wa, wb, xw);
+            load_x(xw, xl, pc.j, 1);
+            decode16(rA1, make_uint2(cA.z, cA.w), B4A, wa);
+            decode16(rB1, make_uint2(cB.z, cB.w), B4B, wb);
+            half_mma(acc[1], wa, wb, xw);
+        } else {
+            // some tile row of the block has escapes: rank them per row (quad
+            // shuffles), decode, patch the escaped weights, multiply
             const bool escA = m0.loA != m0.hiA || (escape_nibbles(cA.x) | escape_nibbles(cA.y) |
                                                    escape_nibbles(cA.z) | escape_nibbles(cA.w)) != 0;
             const bool escB = m0.loB != m0.hiB || (escape_nibbles(cB.x) | escape_nibbles(cB.y) |
                                                    escape_nibbles(cB.z) | escape_nibbles(cB.w)) != 0;
             const unsigned qA = __ballot_sync(0xFFFFFFFFu, escA), qB = __ballot_sync(0xFFFFFFFFu, escB);
+            EscRow eA = {0, 0, 0, 0}, eB = {0, 0, 0, 0};
             if (escA) eA = prepare_row(cA, m0.loA, m0.hiA, mp.n_esc, pr.err, qA, q);
             if (escB) eB = prepare_row(cB, m0.loB, m0.hiB, mp.n_esc, pr.err, qB, q);
-        }
-        const uint32_t B4A = m0.baseA * 0x01010101u, B4B = m0.baseB * 0x01010101u;
-        uint32_t xw[8], wa[8], wb[8];
-        // half 0
-        load_x(xw, xl, pc.j, 0);
-        decode16(rA0, make_uint2(cA.x, cA.y), B4A, wa);
-        decode16(rB0, make_uint2(cB.x, cB.y), B4B, wb);
-        if (any) {
+            load_x(xw, xl, pc.j, 0);
+            decode16(rA0, make_uint2(cA.x, cA.y), B4A, wa);
+            decode16(rB0, make_uint2(cB.x, cB.y), B4B, wb);
             if (eA.has & 1u)
                 fix_chunk(wa, rA0, make_uint2(cA.x, cA.y), m0.baseA, eA.s0, eA.limit, m0.loA, fvA, mp.esc, pr.err, scr);
             if (eB.has & 1u)
                 fix_chunk(wb, rB0, make_uint2(cB.x, cB.y), m0.baseB, eB.s0, eB.limit, m0.loB, fvB, mp.esc, pr.err, scr);
-        }
-        half_mma(acc[0], wa, wb, xw);
-        // half 1
-        load_x(xw, xl, pc.j, 1);
-        decode16(rA1, make_uint2(cA.z, cA.w), B4A, wa);
-        decode16(rB1, make_uint2(cB.z, cB.w), B4B, wb);
-        if (any) {
+            half_mma(acc[0], wa, wb, xw);
+            load_x(xw, xl, pc.j, 1);
+            decode16(rA1, make_uint2(cA.z, cA.w), B4A, wa);
+            decode16(rB1, make_uint2(cB.z, cB.w), B4B, wb);
             if (eA.has & 2u)
                 fix_chunk(wa, rA1, make_uint2(cA.z, cA.w), m0.baseA, eA.s1, eA.limit, m0.loA, fvA, mp.esc, pr.err, scr);
             if (eB.has & 2u)
                 fix_chunk(wb, rB1, make_uint2(cB.z, cB.w), m0.baseB, eB.s1, eB.limit, m0.loB, fvB, mp.esc, pr.err, scr);
+            half_mma(acc[1], wa, wb, xw);
         }
-        half_mma(acc[1], wa, wb, xw);
         if (i + S < nb) advance(pi, pr);
 
         advance(pc, pr);
