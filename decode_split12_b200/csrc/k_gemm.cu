@@ -12,23 +12,24 @@
 // integer-ADD decode feeding tensor-core kernels).
 //
 // One CTA per SM, eighteen warps with fixed roles:
-//   warp 0      TMA producer: per 64-column chunk of a 128-row tile, the raw
-//               plane (128 x 64 bytes), the code plane (128 x 32 bytes) and
-//               the X chunk (M x 64 bf16, 128-byte swizzle) into a ring of
-//               stages, completing on the stage's mbarrier.
-//   warp 1      TMEM owner and MMA issuer: one lane issues four
-//               tcgen05.mma.kind::f16 (K = 16 each) per chunk, A = the
-//               decoded W chunk in shared memory, B = the X chunk, FP32
+//   warp 0      TMA producer: per unit (a 128-row tile x one 128-column tile
+//               column), the raw plane (128 x 128 bytes, 128-byte swizzle),
+//               the code plane (128 x 64 bytes) and the X columns (M x 128
+//               bf16 as two 128-byte-swizzled atoms) into a ring of stages,
+//               completing on the stage's mbarrier.
+//   warp 1      TMEM owner and MMA issuer: one lane issues eight
+//               tcgen05.mma.kind::f16 (K = 16 each) per unit, A = the
+//               decoded W unit in shared memory, B = the X columns, FP32
 //               accumulators in TMEM (128 lanes x M columns), and releases
 //               stages and A buffers with tcgen05.commit.
-//   warps 2..17 decode: each thread owns 16 weights of one row per chunk,
+//   warps 2..17 decode: each thread owns 32 weights of one row per unit,
 //               rebuilds the exact BF16 values (byte-wise base + code ADD,
 //               escapes patched from the escape stream) and stores them in
 //               the canonical K-major 128-byte-swizzled layout the tensor
 //               core reads; then, at the end of each tile, the epilogue:
 //               tcgen05.ld of the accumulators and the stores of Y.
 //
-// Work split (stream-K): the (tile, chunk) units are dealt to the CTAs in
+// Work split (stream-K): the (tile, tile column) units are dealt to the CTAs in
 // equal contiguous ranges.  A tile covered whole by one CTA goes straight to
 // Y; a tile shared by several CTAs is finished by the last of them to
 // arrive, which adds the partials in CTA order (deterministic) from the
@@ -46,18 +47,20 @@ namespace s12 {
 namespace gemm {
 
 constexpr int kRows = 128;         // W rows per tile (UMMA M)
-constexpr int kChunk = 64;         // K columns per chunk (one 128-byte swizzle atom of bf16)
+constexpr int kChunk = 128;        // K columns per unit: one whole tile row
+constexpr int kAtom = 64;          // bf16 columns per 128-byte swizzle atom
 constexpr int kDecodeWarps = 16;
 constexpr int kThreads = 32 * (2 + kDecodeWarps);
-constexpr uint32_t kRawBytes = kRows * kChunk;       // 8 KB
-constexpr uint32_t kCodeBytes = kRows * kChunk / 2;  // 4 KB
-constexpr uint32_t kABytes = kRows * kChunk * 2;     // 16 KB decoded chunk
-constexpr int kABufs = 3;
+constexpr uint32_t kRawBytes = kRows * kChunk;       // 16 KB
+constexpr uint32_t kCodeBytes = kRows * kChunk / 2;  // 8 KB
+constexpr uint32_t kAtomBytes = kRows * kAtom * 2;   // 16 KB: one swizzle atom of the decoded unit
+constexpr uint32_t kABytes = 2 * kAtomBytes;         // 32 KB
+constexpr int kMaxABufs = 2;
 constexpr int kMaxStages = 6;
 
 struct __align__(64) Params {
-    CUtensorMap tm_raw;   // u8 [N][K], box 64 x 128
-    CUtensorMap tm_code;  // u8 [N][K/2], box 32 x 128
+    CUtensorMap tm_raw;   // u8 [N][K], box 128 x 128, 128-byte swizzle
+    CUtensorMap tm_code;  // u8 [N][K/2], box 64 x 128
     CUtensorMap tm_x;     // bf16 [M][K], box 64 x Mp, 128-byte swizzle
     const uint8_t *base;
     const uint32_t *esc_off;
@@ -69,11 +72,13 @@ struct __align__(64) Params {
     uint32_t *cnt;        // workspace: one arrival counter per tile (zero between calls)
     uint32_t *err;
     int N, K, T, M, Mp;   // Mp = M rounded up to a multiple of 16
-    int n_tiles, n_chunks;  // tiles of 128 rows; 64-column chunks per row
+    int n_tiles, n_chunks;  // tiles of 128 rows; 128-column units per row (= tiles per row)
     long long n_units;      // n_tiles * n_chunks
     int stages;
     uint32_t stage_bytes;   // X chunk + raw + code, multiple of 1024
-    uint32_t x_bytes;       // Mp * 128
+    uint32_t x_bytes;       // Mp * 256: the unit's X columns as two swizzle atoms
+    uint32_t x_atom;        // Mp * 128
+    int a_bufs;             // decoded-unit buffers, 1 or 2
     uint32_t tmem_cols;     // power of two >= max(32, Mp)
 };
 
@@ -93,12 +98,42 @@ __device__ __forceinline__ void bar_expect_tx(uint32_t bar, uint32_t bytes) {
 }
 
 // Bounded wait for phase `parity`; false after about a second.
+#ifndef S12_GEMM_WAIT_MODE
+#define S12_GEMM_WAIT_MODE 0
+#endif
+
+__device__ __forceinline__ bool bar_test(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 __device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity) {
-    if (mbar_try_wait(bar, parity)) return true;
+#if S12_GEMM_WAIT_MODE == 1
+    if (bar_test(bar, parity)) return true;
     const long long t0 = clock64();
-    while (!mbar_try_wait_hint(bar, parity, 1000u))  // the thread may sleep up to 1 us per try
+    while (!bar_test(bar, parity))
         if (clock64() - t0 > kWaitCycles) return false;
     return true;
+#elif S12_GEMM_WAIT_MODE == 2
+    if (mbar_try_wait_hint(bar, parity, 20u)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait_hint(bar, parity, 20u))
+        if (clock64() - t0 > kWaitCycles) return false;
+    return true;
+#else
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity))
+        if (clock64() - t0 > kWaitCycles) return false;
+    return true;
+#endif
 }
 
 __device__ __forceinline__ void tma2d(uint32_t dst, const CUtensorMap *tm, int c0, int c1, uint32_t bar,
@@ -233,8 +268,8 @@ __device__ __forceinline__ Layout layout(uint32_t sb, const Params &p) {
     L.full = sb;
     L.empty = sb + 8 * kMaxStages;
     L.a_full = sb + 16 * kMaxStages;
-    L.a_empty = L.a_full + 8 * kABufs;
-    L.acc_full = L.a_empty + 8 * kABufs;
+    L.a_empty = L.a_full + 8 * kMaxABufs;
+    L.acc_full = L.a_empty + 8 * kMaxABufs;
     L.acc_empty = L.acc_full + 8;
     L.done = L.acc_empty + 8;
     L.tmem_slot = L.done + 8;
@@ -261,8 +296,21 @@ __device__ __forceinline__ void fetch_escapes(const Params &p, RowMeta &m) {
 
 // Rows past the end (zeros from the copy engine) read the last row's
 // metadata but report no escapes.
-__device__ __forceinline__ RowMeta load_row_meta(const Params &p, long long unit, int r) {
-    const int tile = static_cast<int>(unit / p.n_chunks), j = static_cast<int>(unit % p.n_chunks) >> 1;
+// A unit's position: 128-row tile and 64-column chunk, advanced without
+// division.
+struct UPos {
+    int tile, chunk;
+};
+
+__device__ __forceinline__ void next(UPos &q, int n_chunks) {
+    if (++q.chunk == n_chunks) {
+        q.chunk = 0;
+        ++q.tile;
+    }
+}
+
+__device__ __forceinline__ RowMeta load_row_meta(const Params &p, UPos q, int r) {
+    const int tile = q.tile, j = q.chunk;  // a unit is one whole tile column
     const int n = tile * kRows + r;
     const size_t t = static_cast<size_t>(min(n, p.N - 1)) * p.T + j;
     RowMeta m;
@@ -274,76 +322,80 @@ __device__ __forceinline__ RowMeta load_row_meta(const Params &p, long long unit
     return m;
 }
 
-// `carry` holds, after a first-half chunk of a tile row with escapes, that
-// half's escape count for the row (all four lanes of the quad); the
-// second-half chunk that follows uses it instead of re-reading the codes.
+// Decode the lane's 32 weights of one tile row (row r of the unit, columns
+// 32*q4 .. +31, as two 16-weight chunks) from the stage into the A buffer,
+// patching escapes.  Called by all 32 lanes; the four lanes of a quad share
+// the row, and escapes are ranked within the row with quad shuffles (chunk
+// order: lane q4 = 0..3, first chunk then second).
 template <bool CHECK>
-__device__ __forceinline__ void decode_piece(const Params &p, uint32_t st_raw, uint32_t st_code, uint32_t abuf,
-                                             int tile, int chunk, int r, int q4, unsigned full_mask,
-                                             const RowMeta &rm, uint32_t &carry, bool carry_ok) {
-    const int n = tile * kRows + r;
-    const int j = chunk >> 1, h = chunk & 1;
-    const int nc = min(n, p.N - 1);
-    const uint32_t base = rm.base, lo = rm.lo, hi = rm.hi;
-    const uint4 raw = lds128(st_raw + r * 64 + q4 * 16);
-    uint2 code = lds64(st_code + r * 32 + q4 * 8);
-    const uint32_t rowa = abuf + static_cast<uint32_t>(r) * 128u, sw = static_cast<uint32_t>(r & 7);
-    uint2 m = make_uint2(0, 0);
+__device__ __forceinline__ void decode_row(const Params &p, uint32_t st_raw, uint32_t st_code, uint32_t abuf,
+                                           int r, int q4, const RowMeta &rm) {
+    const uint32_t sw = static_cast<uint32_t>(r & 7);
+    const uint32_t lo = rm.lo, hi = rm.hi;
+    const uint4 rw0 = lds128(st_raw + r * 128 + (((2u * q4) ^ sw) << 4));  // raw rows are 128-byte swizzled
+    const uint4 rw1 = lds128(st_raw + r * 128 + (((2u * q4 + 1u) ^ sw) << 4));
+    uint4 code = lds128(st_code + r * 64 + 16 * q4);
     bool esc = lo != hi;
+    uint2 m0 = make_uint2(0, 0), m1 = make_uint2(0, 0);
     if (CHECK) {
-        m = make_uint2(escape_nibbles(code.x), escape_nibbles(code.y));
-        if ((m.x | m.y) && !esc) raise_flag(p.err, S12_FLAG_ESC_COUNT);
-        if (base > static_cast<uint32_t>(kMaxBase)) raise_flag(p.err, S12_FLAG_BASE);
+        m0 = make_uint2(escape_nibbles(code.x), escape_nibbles(code.y));
+        m1 = make_uint2(escape_nibbles(code.z), escape_nibbles(code.w));
+        if ((m0.x | m0.y | m1.x | m1.y) && !esc) raise_flag(p.err, S12_FLAG_ESC_COUNT);
+        if (rm.base > static_cast<uint32_t>(kMaxBase)) raise_flag(p.err, S12_FLAG_BASE);
     }
-    const unsigned quads = __ballot_sync(full_mask, esc);
-    uint32_t rank = 0;
+    const unsigned quads = __ballot_sync(0xFFFFFFFFu, esc);
+    uint32_t s0 = 0, s1 = 0;
     if (esc) {
-        if (!CHECK) m = make_uint2(escape_nibbles(code.x), escape_nibbles(code.y));
-        code = make_uint2(clear_escapes(code.x, m.x), clear_escapes(code.y, m.y));  // no carry out of a byte
-        const uint32_t cnt = __popc(m.x) + __popc(m.y);
-        uint32_t incl = cnt;
+        if (!CHECK) {
+            m0 = make_uint2(escape_nibbles(code.x), escape_nibbles(code.y));
+            m1 = make_uint2(escape_nibbles(code.z), escape_nibbles(code.w));
+        }
+        // clear the escape nibbles so base + code never carries out of a byte
+        code = make_uint4(clear_escapes(code.x, m0.x), clear_escapes(code.y, m0.y), clear_escapes(code.z, m1.x),
+                          clear_escapes(code.w, m1.y));
+        const uint32_t n0 = __popc(m0.x) + __popc(m0.y), n = n0 + __popc(m1.x) + __popc(m1.y);
+        uint32_t incl = n;
 #pragma unroll
         for (int d = 1; d < 4; d <<= 1) {
             const uint32_t v = __shfl_up_sync(quads, incl, d, 4);
             if (q4 >= d) incl += v;
         }
-        uint32_t before = 0;  // escapes of this tile row in the first half (columns 0..63)
-        if (h == 1 && carry_ok) {
-            before = carry;
-        } else if (h == 1) {
-            const uint2 c0 = __ldg(reinterpret_cast<const uint2 *>(p.code + static_cast<size_t>(nc) * (p.K / 2) +
-                                                                   static_cast<size_t>(j) * 64 + q4 * 8));
-            uint32_t n0 = __popc(escape_nibbles(c0.x)) + __popc(escape_nibbles(c0.y));
-            n0 += __shfl_xor_sync(quads, n0, 1, 4);
-            n0 += __shfl_xor_sync(quads, n0, 2, 4);
-            before = n0;
-        }
-        const uint32_t total_half = __shfl_sync(quads, incl, 3, 4);
-        if (h == 0) carry = total_half;
-        if (h == 1 && q4 == 0 && before + total_half != hi - lo) raise_flag(p.err, S12_FLAG_ESC_COUNT);
-        if (h == 0 && q4 == 0 && total_half > hi - lo) raise_flag(p.err, S12_FLAG_ESC_COUNT);
-        rank = lo + before + incl - cnt;
+        const uint32_t tot = __shfl_sync(quads, incl, 3, 4);
+        if (q4 == 0 && tot != hi - lo) raise_flag(p.err, S12_FLAG_ESC_COUNT);
+        s0 = lo + incl - n;
+        s1 = s0 + n0;
     }
+    // columns 32*q4 .. +31 lie in atom q4 / 2, at 16-byte pieces pb .. pb + 3
+    const uint32_t row = abuf + static_cast<uint32_t>(q4 >> 1) * kAtomBytes + static_cast<uint32_t>(r) * 128u;
+    const uint32_t pb = 4u * static_cast<uint32_t>(q4 & 1);
+    const uint32_t B4 = rm.base * 0x01010101u;
     uint32_t w[8];
-    decode16(raw, code, base * 0x01010101u, w);
-    sts128(rowa + (((2u * q4) ^ sw) << 4), w[0], w[1], w[2], w[3]);
-    sts128(rowa + (((2u * q4 + 1u) ^ sw) << 4), w[4], w[5], w[6], w[7]);
-    if (esc && (m.x | m.y)) {
+    decode16(rw0, make_uint2(code.x, code.y), B4, w);
+    sts128(row + (((pb + 0u) ^ sw) << 4), w[0], w[1], w[2], w[3]);
+    sts128(row + (((pb + 1u) ^ sw) << 4), w[4], w[5], w[6], w[7]);
+    decode16(rw1, make_uint2(code.z, code.w), B4, w);
+    sts128(row + (((pb + 2u) ^ sw) << 4), w[0], w[1], w[2], w[3]);
+    sts128(row + (((pb + 3u) ^ sw) << 4), w[4], w[5], w[6], w[7]);
+    if (esc) {
         const uint32_t limit = lo <= hi ? static_cast<uint32_t>(hi < p.n_esc ? hi : p.n_esc) : 0u;
-        uint64_t mm = (static_cast<uint64_t>(m.y) << 32) | m.x;
-        uint32_t idx = rank;
-        while (mm) {
-            const int jj = (__ffsll(static_cast<long long>(mm)) - 1) >> 2;  // weight within the piece
-            mm &= mm - 1;
-            uint16_t v = 0;
-            if (idx < limit)
-                v = idx == lo ? static_cast<uint16_t>(rm.fv0)
-                              : (idx == lo + 1 ? static_cast<uint16_t>(rm.fv1) : __ldg(p.esc + idx));
-            else
-                raise_flag(p.err, S12_FLAG_ESC_RANGE);
-            ++idx;
-            const uint32_t kl = static_cast<uint32_t>(q4 * 16 + jj);  // column within the chunk
-            sts16(rowa + ((((kl >> 3) ^ sw)) << 4) + (kl & 7u) * 2u, v);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint2 m = h ? m1 : m0;
+            uint64_t mm = (static_cast<uint64_t>(m.y) << 32) | m.x;
+            uint32_t idx = h ? s1 : s0;
+            while (mm) {
+                const uint32_t jj = static_cast<uint32_t>((__ffsll(static_cast<long long>(mm)) - 1) >> 2);
+                mm &= mm - 1;
+                uint16_t v = 0;
+                if (idx < limit)
+                    v = idx == lo ? static_cast<uint16_t>(rm.fv0)
+                                  : (idx == lo + 1 ? static_cast<uint16_t>(rm.fv1) : __ldg(p.esc + idx));
+                else
+                    raise_flag(p.err, S12_FLAG_ESC_RANGE);
+                ++idx;
+                const uint32_t kl = 8u * pb + 16u * h + jj;  // column within the atom
+                sts16(row + (((kl >> 3) ^ sw) << 4) + (kl & 7u) * 2u, v);
+            }
         }
     }
 }
@@ -436,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             bar_init(L.full + 8 * s, 1);
             bar_init(L.empty + 8 * s, kDecodeWarps + 1);
         }
-        for (int a = 0; a < kABufs; ++a) {
+        for (int a = 0; a < p.a_bufs; ++a) {
             bar_init(L.a_full + 8 * a, kDecodeWarps);
             bar_init(L.a_empty + 8 * a, 1);
         }
@@ -461,8 +513,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             int s = 0;
             uint32_t round = 0;
             long long issued = 0;
-            for (long long u = u0; u < u1; ++u) {
-                const int tile = static_cast<int>(u / p.n_chunks), chunk = static_cast<int>(u % p.n_chunks);
+            UPos q = {static_cast<int>(u0 / p.n_chunks), static_cast<int>(u0 % p.n_chunks)};
+            for (long long u = u0; u < u1; ++u, next(q, p.n_chunks)) {
+                const int tile = q.tile, chunk = q.chunk;
                 if (!bar_wait(L.empty + 8 * s, (round & 1u) ^ 1u)) {
                     raise_flag(p.err, S12_FLAG_TIMEOUT);
                     break;
@@ -470,6 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                 const uint32_t st = L.stages + static_cast<uint32_t>(s) * p.stage_bytes;
                 bar_expect_tx(L.full + 8 * s, p.x_bytes + kRawBytes + kCodeBytes);
                 tma2d(st, &p.tm_x, chunk * kChunk, 0, L.full + 8 * s, pol_x);
+                tma2d(st + p.x_atom, &p.tm_x, chunk * kChunk + kAtom, 0, L.full + 8 * s, pol_x);
                 tma2d(st + p.x_bytes, &p.tm_raw, chunk * kChunk, tile * kRows, L.full + 8 * s, pol_w);
                 tma2d(st + p.x_bytes + kRawBytes, &p.tm_code, chunk * (kChunk / 2), tile * kRows, L.full + 8 * s,
                       pol_w);
@@ -490,8 +544,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             const uint32_t idesc = instr_desc(p.Mp);
             int s = 0, a = 0;
             uint32_t round = 0, around = 0, tiles = 0;
-            for (long long u = u0; u < u1; ++u) {
-                const int chunk = static_cast<int>(u % p.n_chunks);
+            int chunk = static_cast<int>(u0 % p.n_chunks);
+            for (long long u = u0; u < u1; ++u, chunk = (chunk + 1 == p.n_chunks) ? 0 : chunk + 1) {
                 const bool first = (u == u0) || chunk == 0;
                 const bool last = (u + 1 == u1) || chunk == p.n_chunks - 1;
                 bool w = bar_wait(L.full + 8 * s, round & 1u) && bar_wait(L.a_full + 8 * a, around & 1u);
@@ -505,9 +559,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                 const uint32_t xa = L.stages + static_cast<uint32_t>(s) * p.stage_bytes;
                 const uint32_t aa = L.abuf + static_cast<uint32_t>(a) * kABytes;
 #pragma unroll
-                for (int kk = 0; kk < kChunk / 16; ++kk)
-                    umma_bf16(tmem, smem_desc_sw128(aa + kk * 32), smem_desc_sw128(xa + kk * 32), idesc,
-                              (first && kk == 0) ? 0u : 1u);
+                for (int kk = 0; kk < kChunk / 16; ++kk) {
+                    const uint32_t atom = static_cast<uint32_t>(kk >> 2), sub = static_cast<uint32_t>(kk & 3) * 32u;
+                    umma_bf16(tmem, smem_desc_sw128(aa + atom * kAtomBytes + sub),
+                              smem_desc_sw128(xa + atom * p.x_atom + sub), idesc, (first && kk == 0) ? 0u : 1u);
+                }
                 umma_commit(L.empty + 8 * s);
                 umma_commit(L.a_empty + 8 * a);
                 if (last) umma_commit(L.acc_full);
@@ -515,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                     s = 0;
                     ++round;
                 }
-                if (++a == kABufs) {
+                if (++a == p.a_bufs) {
                     a = 0;
                     ++around;
                 }
@@ -533,17 +589,23 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         uint32_t round = 0, around = 0, tiles = 0;
         // the row metadata of the next two units is in flight while a unit is decoded
         RowMeta m0 = {0, 0, 0, 0, 0}, m1 = {0, 0, 0, 0, 0};
+        UPos q = {static_cast<int>(u0 / p.n_chunks), static_cast<int>(u0 % p.n_chunks)};
+        UPos qm = q;  // the unit whose metadata is loaded next
         if (u0 < u1) {
-            m0 = load_row_meta(p, u0, r);
+            m0 = load_row_meta(p, qm, r);
             fetch_escapes(p, m0);
         }
-        if (u0 + 1 < u1) m1 = load_row_meta(p, u0 + 1, r);
-        uint32_t carry = 0;
-        for (long long u = u0; u < u1; ++u) {
-            const int tile = static_cast<int>(u / p.n_chunks), chunk = static_cast<int>(u % p.n_chunks);
+        next(qm, p.n_chunks);
+        if (u0 + 1 < u1) m1 = load_row_meta(p, qm, r);
+        next(qm, p.n_chunks);
+        for (long long u = u0; u < u1; ++u, next(q, p.n_chunks)) {
+            const int tile = q.tile, chunk = q.chunk;
             const bool last = (u + 1 == u1) || chunk == p.n_chunks - 1;
             RowMeta m2 = m1;
-            if (u + 2 < u1) m2 = load_row_meta(p, u + 2, r);
+            if (u + 2 < u1) {
+                m2 = load_row_meta(p, qm, r);
+                next(qm, p.n_chunks);
+            }
             if (u + 1 < u1) fetch_escapes(p, m1);  // m1's offsets arrived during the previous unit
             const bool w = bar_wait(L.full + 8 * s, round & 1u) && bar_wait(L.a_empty + 8 * a, (around & 1u) ^ 1u);
             if (!__all_sync(0xFFFFFFFFu, w)) {
@@ -552,8 +614,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             }
             const uint32_t st = L.stages + static_cast<uint32_t>(s) * p.stage_bytes;
             const uint32_t aa = L.abuf + static_cast<uint32_t>(a) * kABytes;
-            decode_piece<CHECK>(p, st + p.x_bytes, st + p.x_bytes + kRawBytes, aa, tile, chunk, r, q4, 0xFFFFFFFFu, m0,
-                                carry, u > u0);
+            decode_row<CHECK>(p, st + p.x_bytes, st + p.x_bytes + kRawBytes, aa, r, q4, m0);
             m0 = m1;
             m1 = m2;
             // generic-proxy stores must be visible to the tensor core
@@ -567,7 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                 s = 0;
                 ++round;
             }
-            if (++a == kABufs) {
+            if (++a == p.a_bufs) {
                 a = 0;
                 ++around;
             }
@@ -605,7 +666,8 @@ constexpr uint32_t kSmemLimit = 227 * 1024;
 struct Plan {
     int Mp, n_tiles, n_chunks, grid, stages;
     long long n_units;
-    uint32_t x_bytes, stage_bytes, tmem_cols, smem;
+    uint32_t x_bytes, x_atom, stage_bytes, tmem_cols, smem;
+    int a_bufs;
     size_t part_bytes, cnt_bytes;
 };
 
@@ -616,10 +678,17 @@ Plan plan(const s12_view *v, int M, int sms) {
     pl.n_chunks = static_cast<int>(v->cols / gemm::kChunk);
     pl.n_units = static_cast<long long>(pl.n_tiles) * pl.n_chunks;
     pl.grid = static_cast<int>(std::max(1LL, std::min<long long>(sms, pl.n_units)));
-    pl.x_bytes = static_cast<uint32_t>(pl.Mp) * 128u;
+    pl.x_atom = static_cast<uint32_t>(pl.Mp) * 128u;
+    pl.x_bytes = 2 * pl.x_atom;
     pl.stage_bytes = pl.x_bytes + gemm::kRawBytes + gemm::kCodeBytes;
-    const uint32_t fixed = 1024 + 1024 + gemm::kABufs * gemm::kABytes;  // alignment slack, barriers, A buffers
-    pl.stages = static_cast<int>(std::min<uint32_t>(gemm::kMaxStages, (kSmemLimit - fixed) / pl.stage_bytes));
+    // two decoded-unit buffers when two stages still fit beside them, else one
+    pl.a_bufs = gemm::kMaxABufs;
+    uint32_t fixed = 0;
+    for (;; --pl.a_bufs) {
+        fixed = 1024 + 1024 + static_cast<uint32_t>(pl.a_bufs) * gemm::kABytes;  // slack, barriers, A buffers
+        pl.stages = static_cast<int>(std::min<uint32_t>(gemm::kMaxStages, (kSmemLimit - fixed) / pl.stage_bytes));
+        if (pl.stages >= 2 || pl.a_bufs == 1) break;
+    }
     pl.smem = fixed + static_cast<uint32_t>(pl.stages) * pl.stage_bytes;
     uint32_t cols = 32;
     while (cols < static_cast<uint32_t>(pl.Mp)) cols <<= 1;
@@ -648,10 +717,10 @@ int launch_gemm(const s12_view *v, const uint16_t *x, int M, float *y, void *ws,
     if (pl.stages < 2) return S12_ERR_SHAPE;
     gemm::Params p = {};
     const uint64_t N = v->rows, K = v->cols;
-    if (make_tmap_u8_2d(&p.tm_raw, v->raw, K, N, K, gemm::kChunk, gemm::kRows, false) != S12_OK) return S12_ERR_CUDA;
+    if (make_tmap_u8_2d(&p.tm_raw, v->raw, K, N, K, gemm::kChunk, gemm::kRows, true) != S12_OK) return S12_ERR_CUDA;
     if (make_tmap_u8_2d(&p.tm_code, v->code, K / 2, N, K / 2, gemm::kChunk / 2, gemm::kRows, false) != S12_OK)
         return S12_ERR_CUDA;
-    if (make_tmap_bf16_2d(&p.tm_x, x, K, static_cast<uint64_t>(M), K * 2, gemm::kChunk, static_cast<uint32_t>(pl.Mp),
+    if (make_tmap_bf16_2d(&p.tm_x, x, K, static_cast<uint64_t>(M), K * 2, gemm::kAtom, static_cast<uint32_t>(pl.Mp),
                           true) != S12_OK)
         return S12_ERR_CUDA;
     p.base = v->base;
@@ -674,6 +743,8 @@ int launch_gemm(const s12_view *v, const uint16_t *x, int M, float *y, void *ws,
     p.stages = pl.stages;
     p.stage_bytes = pl.stage_bytes;
     p.x_bytes = pl.x_bytes;
+    p.x_atom = pl.x_atom;
+    p.a_bufs = pl.a_bufs;
     p.tmem_cols = pl.tmem_cols;
     auto kern = err ? gemm::gemm_tc_kernel<true> : gemm::gemm_tc_kernel<false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem) != cudaSuccess)
