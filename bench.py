@@ -443,6 +443,10 @@ def run_llama8b(args, world, rank):
         del layer.w_dev
         torch.cuda.empty_cache()
         extra["gemm_70b_mlp_tcgen05"] = gemm_extras(world)
+    if not args.no_decode:
+        extra["decode_escape_stress"] = decode_extras(world)
+    if not args.no_stack:
+        extra["whole_stack"] = stack_extras(world)
     del ge
     traffic = load_traffic("gemv_tma_kernel", f"llama8b_b{args.batch}")
     out = {
@@ -532,6 +536,150 @@ def gemm_extras(world, steps: int = 40):
         out[f"{name}_{n}x{k}"] = {"container_bytes": cbytes, **res}
         del wd, blob
         torch.cuda.empty_cache()
+    return out
+
+
+def decode_extras(world, steps: int = 30):
+    """Standalone decode on the escape-rate stress tensors (8192 x 8192,
+    exactly 0.03 %, 0.23 %, 2 % and 10 % escapes at uniform positions):
+    throughput and a bit-exact check of the whole output against the source
+    tensor on the device."""
+    import torch
+
+    from decode_split12_b200 import s12
+    hbm, _, _, _ = load_peaks()
+    out = {}
+    for rate in wl.ESCAPE_RATES:
+        w, n_planted = wl.escape_stress(rate, 0)
+        wd = dev16(w)
+        del w
+        blob = s12.s12_encode(wd)
+        view = s12.s12_open(blob)
+        dst = torch.empty_like(wd)
+        flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+        g = capture(lambda: s12.s12_decode(view, dst, err_flag=flag))
+        for _ in range(3):
+            g.replay()
+        t = time_graph(g, steps, world) / steps
+        exact = bool(torch.equal(dst, wd)) and int(flag.item()) == 0
+        n, nt = int(view.rows * view.cols), int(view.n_tiles)
+        alg = n * 3 // 2 + nt * 5 + 4 + 2 * int(view.n_esc) + 2 * n
+        out[f"{rate * 100:g}%"] = {"n_esc": int(view.n_esc), "planted": n_planted, "bit_exact": exact,
+                                   "us": round(t * 1e6, 2), "hbm_GBs": round(alg / t / 1e9, 1),
+                                   "hbm_frac": round(alg / t / 1e9 / hbm, 4),
+                                   "bf16_out_GBs": round(2 * n / t / 1e9, 1)}
+        del g, wd, blob, dst
+        torch.cuda.empty_cache()
+    return out
+
+
+def _student_t_gpu(rows: int, cols: int, gen):
+    """Student-t(5) scaled to std 1/sqrt(cols), drawn on the device: t = z /
+    sqrt(chi2_5 / 5) with chi2_5 = 2 * Gamma(2.5); rounded to BF16."""
+    import torch
+    z = torch.randn(rows, cols, generator=gen, device="cuda")
+    gam = torch._standard_gamma(torch.full((rows, cols), 2.5, device="cuda"), generator=gen)
+    t = z / torch.sqrt(2.0 * gam / 5.0)
+    del z, gam
+    return (t * (1.0 / math.sqrt(5.0 / 3.0) / math.sqrt(cols))).to(torch.bfloat16).view(torch.int16)
+
+
+def stack_extras(world, layers: int = 32, steps: int = 10):
+    """Whole-stack weight streaming: `layers` independent 8B-style layers
+    (layer l drawn with seed l) resident as Split12 containers, one grouped
+    launch per layer (its seven GEMVs), one pass = all layers; B = 1 and 8.
+    Plus an 8-expert MoE block (gate, up 14336x4096, down 4096x14336 per
+    expert) with top-2 routing of 64 tokens: experts with >= 9 tokens use the
+    skinny GEMM (rows padded to 16), the rest the GEMV."""
+    import torch
+
+    from decode_split12_b200 import s12
+    hbm, _, _, _ = load_peaks()
+    names = list(wl.LLAMA8B_SHAPES)
+    blobs, views = [], []
+    for layer in range(layers):
+        gen = torch.Generator(device="cuda").manual_seed(layer)
+        lv = []
+        for n in names:
+            r, c = wl.LLAMA8B_SHAPES[n]
+            wd = _student_t_gpu(r, c, gen)
+            b = s12.s12_encode(wd)
+            del wd
+            blobs.append(b)
+            lv.append(s12.s12_open(b))
+        views.append(lv)
+    torch.cuda.empty_cache()
+    weights = layers * sum(r * c for r, c in wl.LLAMA8B_SHAPES.values())
+    cbytes = sum(int(v.container_bytes) for lv in views for v in lv)
+    ws = torch.zeros(s12.s12_gemv_multi_ws_bytes(views[0], 8), dtype=torch.uint8, device="cuda")
+    out = {"layers": layers, "weights": weights, "container_bytes": cbytes}
+    for B in (1, 8):
+        xs = [dev16(wl.activations(B, wl.LLAMA8B_SHAPES[n][1], B, 3000 + i)) for i, n in enumerate(names)]
+        ys = [torch.empty((B, wl.LLAMA8B_SHAPES[n][0]), dtype=torch.float32, device="cuda") for n in names]
+
+        def step():
+            for lv in views:
+                s12.s12_gemv_multi(lv, xs, ys, ws=ws)
+
+        g = capture(step)
+        for _ in range(3):
+            g.replay()
+        t = time_graph(g, steps, world) / steps
+        out[f"B{B}"] = {"ms_per_pass": round(t * 1e3, 3), "ms_per_token": round(t * 1e3 / B, 3),
+                        "effective_bf16_GBs": round(2 * weights / t / 1e9, 1),
+                        "hbm_frac": round(cbytes / t / 1e9 / hbm, 4), "launches_per_pass": layers}
+        del g
+    del blobs, views
+    torch.cuda.empty_cache()
+    # MoE block
+    route = wl.moe_routing(64, 8, 2, 0)
+    experts = []
+    gen = torch.Generator(device="cuda").manual_seed(1000)
+    for e in range(8):
+        ev = {}
+        for n, (r, c) in wl.MOE_SHAPES.items():
+            wd = _student_t_gpu(r, c, gen)
+            b = s12.s12_encode(wd)
+            del wd
+            ev[n] = (b, s12.s12_open(b))
+        experts.append(ev)
+    counts = [int((route == e).any(axis=1).sum()) for e in range(8)]
+    calls = []
+    for e, m in enumerate(counts):
+        if m == 0:
+            continue
+        for n, (r, c) in wl.MOE_SHAPES.items():
+            v = experts[e][n][1]
+            if m >= 9:
+                mp = max(16, m)
+                x = dev16(wl.activations(mp, c, e, 4000 + 10 * e + len(calls)))
+                y = torch.empty((mp, r), dtype=torch.float32, device="cuda")
+                gws = torch.zeros(s12.s12_gemm_ws_bytes(v, mp), dtype=torch.uint8, device="cuda")
+                calls.append(("gemm", v, x, y, gws))
+            else:
+                x = dev16(wl.activations(m, c, e, 4000 + 10 * e + len(calls)))
+                y = torch.empty((m, r), dtype=torch.float32, device="cuda")
+                gws = torch.zeros(s12.s12_gemv_ws_bytes(v, m), dtype=torch.uint8, device="cuda")
+                calls.append(("gemv", v, x, y, gws))
+
+    def moe():
+        for kind, v, x, y, gws in calls:
+            if kind == "gemm":
+                s12.s12_gemm_skinny(v, x, y, ws=gws)
+            else:
+                s12.s12_gemv(v, x, y, ws=gws)
+
+    g = capture(moe)
+    for _ in range(3):
+        g.replay()
+    t = time_graph(g, steps, world) / steps
+    moe_bytes = sum(int(experts[e][n][1].container_bytes) for e in range(8) if counts[e] for n in wl.MOE_SHAPES)
+    out["moe_8x_top2_64_tokens"] = {"tokens_per_expert": counts, "us": round(t * 1e6, 2),
+                                    "us_per_token": round(t * 1e6 / 64, 3),
+                                    "hbm_frac": round(moe_bytes / t / 1e9 / hbm, 4),
+                                    "calls": [c[0] for c in calls]}
+    del g, experts, calls
+    torch.cuda.empty_cache()
     return out
 
 
@@ -656,6 +804,8 @@ def main(argv=None):
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-gemm", action="store_true", help="skip the skinny-GEMM extras")
+    ap.add_argument("--no-decode", action="store_true", help="skip the standalone-decode extras")
+    ap.add_argument("--no-stack", action="store_true", help="skip the whole-stack extras")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
