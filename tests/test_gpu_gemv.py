@@ -198,3 +198,70 @@ def test_gemv_multi_rejects_bad_groups(s12):
     x = to_dev(wl.activations(1, 256, 0))
     with pytest.raises(s12.S12Error):
         s12.s12_gemv_multi([v] * 9, [x] * 9)
+
+
+def test_gemv_top_of_range_bases(s12, oracle):
+    """Tiles whose window sits at the top of the BF16 range (base 240 or 241,
+    where base + 15 is an Inf/NaN exponent or carries out of the byte) with
+    escapes below the window.  x is scaled down so that no product or sum
+    leaves the FP32 range; the result matches the FP64 oracle."""
+    g = wl.rng_for(21, 0)
+    w = wl.normal_with_outliers(64, 1024, 0.02, 0.0, 21)
+    for r in range(64):
+        e = g.integers(241, 255, size=1024)                     # window [240, 254] or [241, 255]
+        e[g.choice(1024, 6, replace=False)] = g.integers(100, 130, size=6)   # escapes
+        w[r] = ((g.integers(0, 2, 1024) << 15) | (e << 7) | g.integers(0, 128, 1024)).astype(np.uint16)
+    x = wl.to_bf16_bits(wl.rng_for(22, 0).standard_normal((2, 1024)).astype(np.float32) * np.float32(2.0 ** -120))
+    flag = new_flag()
+    _, _, y = _gemv(s12, w, x, flag)
+    yr, sr = oracle.gemv_f64(oracle.encode(w), x)
+    assert np.isfinite(y).all()
+    assert_within_tolerance(y, yr, sr)
+    assert int(flag.item()) == 0
+
+
+@pytest.mark.parametrize("B", [1, 5, 8])
+def test_gemv_huge_activations_at_escapes(s12, oracle, B):
+    """Zero weights (always escapes, below every window) at six columns in
+    40 of the rows, and x 2^40 times larger at exactly those columns.  The
+    true sums of those rows are near 30 while any finite placeholder value
+    at the escapes would give products near 1e12 (FP32 spacing 2^17 there),
+    so a kernel must use the exact escaped values inside the product, not
+    add a placeholder and cancel it later.  Checked against the FP64 oracle
+    within the usual tolerance, and the error word stays clear."""
+    R, K = 96, 2048
+    w = wl.normal_with_outliers(R, K, 0.02, 0.0, 31)
+    g = wl.rng_for(31, 1)
+    hot = g.choice(K, 6, replace=False)
+    rows = g.choice(R, 40, replace=False)
+    w[np.ix_(rows, hot)] = 0          # +0.0 in bf16: exponent 0, an escape
+    xf = g.standard_normal((B, K)).astype(np.float32)
+    xf[:, hot] *= np.float32(2.0 ** 40)
+    x = wl.to_bf16_bits(xf)
+    flag = new_flag()
+    _, _, y = _gemv(s12, w, x, flag)
+    yr, sr = oracle.gemv_f64(oracle.encode(w), x)
+    assert np.isfinite(y).all()
+    assert_within_tolerance(y, yr, sr)
+    assert int(flag.item()) == 0
+
+
+def test_gemv_inf_activation_at_escape(s12, oracle):
+    """x = +Inf at a column where one row has a zero weight (an escape) and
+    the others ordinary weights: the zero row's exact result is NaN
+    (0 * Inf), the rows with a nonzero weight there give +-Inf with the
+    weight's sign (no escape may be replaced by a finite value there)."""
+    R, K = 32, 512
+    w = wl.normal_with_outliers(R, K, 0.02, 0.0, 41)
+    col = 77
+    w[5, col] = 0
+    xf = wl.rng_for(41, 1).standard_normal((1, K)).astype(np.float32)
+    xf[0, col] = np.inf
+    x = wl.to_bf16_bits(xf)
+    _, _, y = _gemv(s12, w, x, new_flag())
+    wf = (w.astype(np.uint32) << 16).view(np.float32)
+    for r in range(R):
+        if r == 5:
+            assert np.isnan(y[0, r])
+        else:
+            assert y[0, r] == (np.inf if wf[r, col] > 0 else -np.inf), r
