@@ -655,15 +655,15 @@ def stack_extras(world, layers: int = 32, steps: int = 10):
                 x = dev16(wl.activations(mp, c, e, 4000 + 10 * e + len(calls)))
                 y = torch.empty((mp, r), dtype=torch.float32, device="cuda")
                 gws = torch.zeros(s12.s12_gemm_ws_bytes(v, mp), dtype=torch.uint8, device="cuda")
-                calls.append(("gemm", v, x, y, gws))
+                calls.append(("gemm", v, x, y, gws, n))
             else:
                 x = dev16(wl.activations(m, c, e, 4000 + 10 * e + len(calls)))
                 y = torch.empty((m, r), dtype=torch.float32, device="cuda")
                 gws = torch.zeros(s12.s12_gemv_ws_bytes(v, m), dtype=torch.uint8, device="cuda")
-                calls.append(("gemv", v, x, y, gws))
+                calls.append(("gemv", v, x, y, gws, n))
 
     def moe():
-        for kind, v, x, y, gws in calls:
+        for kind, v, x, y, gws, _ in calls:
             if kind == "gemm":
                 s12.s12_gemm_skinny(v, x, y, ws=gws)
             else:
@@ -678,7 +678,43 @@ def stack_extras(world, layers: int = 32, steps: int = 10):
                                     "us_per_token": round(t * 1e6 / 64, 3),
                                     "hbm_frac": round(moe_bytes / t / 1e9 / hbm, 4),
                                     "calls": [c[0] for c in calls]}
-    del g, experts, calls
+    del g
+    # the same block as grouped launches, in the order its data flow allows:
+    # every expert's gate and up in one launch, every expert's down in another
+    # (experts with fewer than 9 tokens, if any, as grouped GEMVs beside them)
+    stages = []
+    for names in (("gate", "up"), ("down",)):
+        gv, gx, gy, vv, vx, vy = [], [], [], [], [], []
+        for kind, v, x, y, _, n in calls:
+            if n not in names:
+                continue
+            if kind == "gemm":
+                gv.append(v), gx.append(x), gy.append(y)
+            else:
+                vv.append(v), vx.append(x), vy.append(y)
+        gws = torch.zeros(max(256, s12.s12_gemm_multi_ws_bytes(gv, [x.shape[0] for x in gx])) if gv else 256,
+                          dtype=torch.uint8, device="cuda")
+        vws = [torch.zeros(max(256, s12.s12_gemv_multi_ws_bytes([v], x.shape[0])), dtype=torch.uint8,
+                           device="cuda") for v, x in zip(vv, vx)]
+        stages.append((gv, gx, gy, gws, vv, vx, vy, vws))
+
+    def moe_grouped():
+        for gv, gx, gy, gws, vv, vx, vy, vws in stages:
+            if gv:
+                s12.s12_gemm_skinny_multi(gv, gx, gy, ws=gws)
+            for v, x, y, w_ in zip(vv, vx, vy, vws):
+                s12.s12_gemv(v, x, y, ws=w_)
+
+    g = capture(moe_grouped)
+    for _ in range(3):
+        g.replay()
+    t = time_graph(g, steps, world) / steps
+    out["moe_8x_top2_64_tokens_grouped"] = {
+        "us": round(t * 1e6, 2), "us_per_token": round(t * 1e6 / 64, 3),
+        "hbm_frac": round(moe_bytes / t / 1e9 / hbm, 4),
+        "launches": sum((1 if st[0] else 0) + len(st[4]) for st in stages),
+        "grouping": "one s12_gemm_skinny_multi over all experts' gate and up, one over all experts' down"}
+    del g, experts, calls, stages
     torch.cuda.empty_cache()
     return out
 

@@ -57,23 +57,34 @@ constexpr uint32_t kAtomBytes = kRows * kAtom * 2;   // 16 KB: one swizzle atom 
 constexpr uint32_t kABytes = 2 * kAtomBytes;         // 32 KB
 constexpr int kMaxABufs = 2;
 constexpr int kMaxStages = 6;
+constexpr int kMaxProblems = S12_GEMM_MAX_PROBLEMS;
 
-struct __align__(64) Params {
+// One matrix of a call (a grouped call has several, with their own shapes,
+// token rows and outputs).
+struct __align__(64) Problem {
     CUtensorMap tm_raw;   // u8 [N][K], box 128 x 128, 128-byte swizzle
     CUtensorMap tm_code;  // u8 [N][K/2], box 64 x 128
-    CUtensorMap tm_x;     // bf16 [M][K], box 64 x Mp, 128-byte swizzle
+    CUtensorMap tm_x;     // bf16 [M][K], box 64 x Mp, 128-byte swizzle (rows >= M read as 0)
     const uint8_t *base;
     const uint32_t *esc_off;
     const uint16_t *esc;
-    const uint8_t *code;  // the code plane in global memory (escape ranking)
     uint64_t n_esc;
-    float *y;             // M x N fp32
+    float *y;               // M x N fp32
+    long long unit0;        // first unit of this matrix in the call's numbering
+    int N, K, T, M;
+    int n_tiles, n_chunks;  // tiles of 128 rows; 128-column units per row (= tiles per row)
+    int tile0;              // first tile of this matrix in the call's numbering (counters)
+};
+
+template <int NP>
+struct __align__(64) Params {
+    Problem prob[NP];
     float *part;          // workspace: [grid][2][Mp][kRows] partial tiles
     uint32_t *cnt;        // workspace: one arrival counter per tile (zero between calls)
     uint32_t *err;
-    int N, K, T, M, Mp;   // Mp = M rounded up to a multiple of 16
-    int n_tiles, n_chunks;  // tiles of 128 rows; 128-column units per row (= tiles per row)
-    long long n_units;      // n_tiles * n_chunks
+    int n_problems;
+    int Mp;               // the largest M of the call rounded up to a multiple of 16
+    long long n_units;    // all matrices' units
     int stages;
     uint32_t stage_bytes;   // X chunk + raw + code, multiple of 1024
     uint32_t x_bytes;       // Mp * 256: the unit's X columns as two swizzle atoms
@@ -263,7 +274,8 @@ struct Layout {
     uint32_t stages, abuf;                                        // data regions
 };
 
-__device__ __forceinline__ Layout layout(uint32_t sb, const Params &p) {
+template <int NP>
+__device__ __forceinline__ Layout layout(uint32_t sb, const Params<NP> &p) {
     Layout L;
     L.full = sb;
     L.empty = sb + 8 * kMaxStages;
@@ -286,9 +298,10 @@ __device__ __forceinline__ Layout layout(uint32_t sb, const Params &p) {
 struct RowMeta {
     uint32_t base, lo, hi;
     uint32_t fv0, fv1;  // the tile row's first two escape values (fetched one unit ahead)
+    int pi;             // the matrix the unit belongs to
 };
 
-__device__ __forceinline__ void fetch_escapes(const Params &p, RowMeta &m) {
+__device__ __forceinline__ void fetch_escapes(const Problem &p, RowMeta &m) {
     m.fv0 = m.fv1 = 0;
     if (m.lo < m.hi && m.lo < p.n_esc) m.fv0 = __ldg(p.esc + m.lo);
     if (m.lo + 1 < m.hi && m.lo + 1 < p.n_esc) m.fv1 = __ldg(p.esc + m.lo + 1);
@@ -296,20 +309,42 @@ __device__ __forceinline__ void fetch_escapes(const Params &p, RowMeta &m) {
 
 // Rows past the end (zeros from the copy engine) read the last row's
 // metadata but report no escapes.
-// A unit's position: 128-row tile and 64-column chunk, advanced without
-// division.
+// A unit's position: matrix, 128-row tile and tile column, advanced without
+// division (units run tile-major within a matrix, matrices in call order).
 struct UPos {
-    int tile, chunk;
+    int p, tile, chunk;
 };
 
-__device__ __forceinline__ void next(UPos &q, int n_chunks) {
-    if (++q.chunk == n_chunks) {
+// (with one matrix, NP = 1, the matrix index stays a compile-time 0)
+template <int NP>
+__device__ __forceinline__ void next(UPos &q, const Params<NP> &P) {
+    if (++q.chunk == P.prob[NP == 1 ? 0 : q.p].n_chunks) {
         q.chunk = 0;
         ++q.tile;
+        if (NP > 1 && q.tile == P.prob[q.p].n_tiles) {
+            q.tile = 0;
+            if (q.p + 1 < P.n_problems) ++q.p;
+        }
     }
 }
 
-__device__ __forceinline__ RowMeta load_row_meta(const Params &p, UPos q, int r) {
+// Position of unit u (one division, once per CTA).
+template <int NP>
+__device__ __forceinline__ UPos locate(const Params<NP> &P, long long u) {
+    int i = 0;
+    if (NP > 1)
+        while (i + 1 < P.n_problems && u >= P.prob[i + 1].unit0) ++i;
+    const long long lu = u - P.prob[i].unit0;
+    UPos q;
+    q.p = i;
+    q.tile = static_cast<int>(lu / P.prob[i].n_chunks);
+    q.chunk = static_cast<int>(lu - static_cast<long long>(q.tile) * P.prob[i].n_chunks);
+    return q;
+}
+
+template <int NP>
+__device__ __forceinline__ RowMeta load_row_meta(const Params<NP> &P, UPos q, int r) {
+    const Problem &p = P.prob[q.p];
     const int tile = q.tile, j = q.chunk;  // a unit is one whole tile column
     const int n = tile * kRows + r;
     const size_t t = static_cast<size_t>(min(n, p.N - 1)) * p.T + j;
@@ -319,6 +354,7 @@ __device__ __forceinline__ RowMeta load_row_meta(const Params &p, UPos q, int r)
     m.hi = __ldg(p.esc_off + t + 1);
     if (n >= p.N) m.hi = m.lo;
     m.fv0 = m.fv1 = 0;
+    m.pi = q.p;
     return m;
 }
 
@@ -328,8 +364,8 @@ __device__ __forceinline__ RowMeta load_row_meta(const Params &p, UPos q, int r)
 // the row, and escapes are ranked within the row with quad shuffles (chunk
 // order: lane q4 = 0..3, first chunk then second).
 template <bool CHECK>
-__device__ __forceinline__ void decode_row(const Params &p, uint32_t st_raw, uint32_t st_code, uint32_t abuf,
-                                           int r, int q4, const RowMeta &rm) {
+__device__ __forceinline__ void decode_row(const Problem &p, uint32_t *err, uint32_t st_raw, uint32_t st_code,
+                                           uint32_t abuf, int r, int q4, const RowMeta &rm) {
     const uint32_t sw = static_cast<uint32_t>(r & 7);
     const uint32_t lo = rm.lo, hi = rm.hi;
     const uint4 rw0 = lds128(st_raw + r * 128 + (((2u * q4) ^ sw) << 4));  // raw rows are 128-byte swizzled
@@ -340,8 +376,8 @@ __device__ __forceinline__ void decode_row(const Params &p, uint32_t st_raw, uin
     if (CHECK) {
         m0 = make_uint2(escape_nibbles(code.x), escape_nibbles(code.y));
         m1 = make_uint2(escape_nibbles(code.z), escape_nibbles(code.w));
-        if ((m0.x | m0.y | m1.x | m1.y) && !esc) raise_flag(p.err, S12_FLAG_ESC_COUNT);
-        if (rm.base > static_cast<uint32_t>(kMaxBase)) raise_flag(p.err, S12_FLAG_BASE);
+        if ((m0.x | m0.y | m1.x | m1.y) && !esc) raise_flag(err, S12_FLAG_ESC_COUNT);
+        if (rm.base > static_cast<uint32_t>(kMaxBase)) raise_flag(err, S12_FLAG_BASE);
     }
     const unsigned quads = __ballot_sync(0xFFFFFFFFu, esc);
     uint32_t s0 = 0, s1 = 0;
@@ -361,7 +397,7 @@ __device__ __forceinline__ void decode_row(const Params &p, uint32_t st_raw, uin
             if (q4 >= d) incl += v;
         }
         const uint32_t tot = __shfl_sync(quads, incl, 3, 4);
-        if (q4 == 0 && tot != hi - lo) raise_flag(p.err, S12_FLAG_ESC_COUNT);
+        if (q4 == 0 && tot != hi - lo) raise_flag(err, S12_FLAG_ESC_COUNT);
         s0 = lo + incl - n;
         s1 = s0 + n0;
     }
@@ -391,7 +427,7 @@ __device__ __forceinline__ void decode_row(const Params &p, uint32_t st_raw, uin
                     v = idx == lo ? static_cast<uint16_t>(rm.fv0)
                                   : (idx == lo + 1 ? static_cast<uint16_t>(rm.fv1) : __ldg(p.esc + idx));
                 else
-                    raise_flag(p.err, S12_FLAG_ESC_RANGE);
+                    raise_flag(err, S12_FLAG_ESC_RANGE);
                 ++idx;
                 const uint32_t kl = 8u * pb + 16u * h + jj;  // column within the atom
                 sts16(row + (((kl >> 3) ^ sw) << 4) + (kl & 7u) * 2u, v);
@@ -406,21 +442,27 @@ __device__ __forceinline__ void decode_row(const Params &p, uint32_t st_raw, uin
 namespace s12 {
 namespace gemm {
 
-// Epilogue for tile `tile` (the accumulators are final for this CTA's part
-// of it): store Y directly, or hand the partial to the stream-K fix-up.
-// Run by the 512 decode threads (warps 2..17); ew = warp - 2.
-__device__ __forceinline__ void epilogue(const Params &p, uint32_t tmem, const Layout &L, int tile, long long u0,
-                                         long long u1, int ew, int lane) {
+// Epilogue for tile `tile` of matrix pr (the accumulators are final for this
+// CTA's part of it): store Y directly, or hand the partial to the stream-K
+// fix-up.  gtile is the tile's index in the call's numbering (its counter),
+// [t0, t1) its units.  A CTA's first tile uses partial slot 0, any later one
+// slot 1; the CTA whose range starts at unit cs therefore used slot 0 for
+// this tile exactly when cs >= t0.  Run by the 512 decode threads (warps
+// 2..17); ew = warp - 2.
+template <int NP>
+__device__ __forceinline__ void epilogue(const Params<NP> &p, const Problem &pr, uint32_t tmem, const Layout &L,
+                                         int tile, int gtile, long long t0, long long u0, long long u1, int ew,
+                                         int lane) {
     const int warp = ew + 2;
     const int quad = warp & 3;                 // TMEM lanes 32*quad .. +31 are this warp's
     const int row = quad * 32 + lane;          // row within the tile
     const int n = tile * kRows + row;
     const int part_cols = p.Mp / 4, c_begin = (ew >> 2) * part_cols;  // four warps share a lane quadrant
     const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-    const long long t0 = static_cast<long long>(tile) * p.n_chunks, t1 = t0 + p.n_chunks;
+    const long long t1 = t0 + pr.n_chunks;
     const bool whole = t0 >= u0 && t1 <= u1;
     const int cta = blockIdx.x;
-    const int slot = (tile == static_cast<int>(u0 / p.n_chunks)) ? 0 : 1;
+    const int slot = u0 >= t0 ? 0 : 1;
     float *mine = p.part + (static_cast<size_t>(cta) * 2 + slot) * static_cast<size_t>(p.Mp) * kRows;
     for (int c = c_begin; c < c_begin + part_cols; c += 4) {
         uint32_t v[4];
@@ -430,7 +472,7 @@ __device__ __forceinline__ void epilogue(const Params &p, uint32_t tmem, const L
         for (int i = 0; i < 4; ++i) {
             const int m = c + i;
             if (whole) {
-                if (m < p.M && n < p.N) p.y[static_cast<size_t>(m) * p.N + n] = __uint_as_float(v[i]);
+                if (m < pr.M && n < pr.N) pr.y[static_cast<size_t>(m) * pr.N + n] = __uint_as_float(v[i]);
             } else {
                 __stcg(mine + static_cast<size_t>(m) * kRows + row, __uint_as_float(v[i]));
             }
@@ -448,7 +490,7 @@ __device__ __forceinline__ void epilogue(const Params &p, uint32_t tmem, const L
         uint32_t n_contrib = 0;
         for (long long c = cf; c <= cl; ++c)
             if (unit_start(c, n_units, grid) < unit_start(c + 1, n_units, grid)) ++n_contrib;
-        const uint32_t prev = atomicAdd(p.cnt + tile, 1u);
+        const uint32_t prev = atomicAdd(p.cnt + gtile, 1u);
         asm volatile("st.shared.u32 [%0], %1;" ::"r"(L.xchg), "r"(prev + 1 == n_contrib ? 1u : 0u) : "memory");
     }
     asm volatile("bar.sync 1, %0;" ::"n"(32 * kDecodeWarps) : "memory");
@@ -462,19 +504,19 @@ __device__ __forceinline__ void epilogue(const Params &p, uint32_t tmem, const L
         for (long long c = cf; c <= cl; ++c) {
             const long long cs = unit_start(c, n_units, grid);
             if (cs >= unit_start(c + 1, n_units, grid)) continue;
-            const int sl = (tile == static_cast<int>(cs / p.n_chunks)) ? 0 : 1;
+            const int sl = cs >= t0 ? 0 : 1;
             s += __ldcg(p.part + (static_cast<size_t>(c) * 2 + sl) * static_cast<size_t>(p.Mp) * kRows +
                         static_cast<size_t>(idx));
         }
         const int nn = tile * kRows + r;
-        if (m < p.M && nn < p.N) p.y[static_cast<size_t>(m) * p.N + nn] = s;
+        if (m < pr.M && nn < pr.N) pr.y[static_cast<size_t>(m) * pr.N + nn] = s;
     }
     asm volatile("bar.sync 1, %0;" ::"n"(32 * kDecodeWarps) : "memory");
-    if (ew == 0 && lane == 0) atomicExch(p.cnt + tile, 0u);
+    if (ew == 0 && lane == 0) atomicExch(p.cnt + gtile, 0u);
 }
 
-template <bool CHECK>
-__global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ Params p) {
+template <bool CHECK, int NP>
+__global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ Params<NP> p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t sb = (smem_addr(smem_raw) + 1023u) & ~1023u;
     const Layout L = layout(sb, p);
@@ -506,6 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     tc_fence_after();
     uint32_t tmem;
     asm volatile("ld.shared.u32 %0, [%1];" : "=r"(tmem) : "r"(L.tmem_slot) : "memory");
+    const UPos q0 = u0 < u1 ? locate(p, u0) : UPos{0, 0, 0};
     if (warp == 0) {
         // ---- TMA producer
         if (lane == 0) {
@@ -513,8 +556,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             int s = 0;
             uint32_t round = 0;
             long long issued = 0;
-            UPos q = {static_cast<int>(u0 / p.n_chunks), static_cast<int>(u0 % p.n_chunks)};
-            for (long long u = u0; u < u1; ++u, next(q, p.n_chunks)) {
+            UPos q = q0;
+            for (long long u = u0; u < u1; ++u, next(q, p)) {
+                const Problem &pr = p.prob[q.p];
                 const int tile = q.tile, chunk = q.chunk;
                 if (!bar_wait(L.empty + 8 * s, (round & 1u) ^ 1u)) {
                     raise_flag(p.err, S12_FLAG_TIMEOUT);
@@ -522,10 +566,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                 }
                 const uint32_t st = L.stages + static_cast<uint32_t>(s) * p.stage_bytes;
                 bar_expect_tx(L.full + 8 * s, p.x_bytes + kRawBytes + kCodeBytes);
-                tma2d(st, &p.tm_x, chunk * kChunk, 0, L.full + 8 * s, pol_x);
-                tma2d(st + p.x_atom, &p.tm_x, chunk * kChunk + kAtom, 0, L.full + 8 * s, pol_x);
-                tma2d(st + p.x_bytes, &p.tm_raw, chunk * kChunk, tile * kRows, L.full + 8 * s, pol_w);
-                tma2d(st + p.x_bytes + kRawBytes, &p.tm_code, chunk * (kChunk / 2), tile * kRows, L.full + 8 * s,
+                tma2d(st, &pr.tm_x, chunk * kChunk, 0, L.full + 8 * s, pol_x);
+                tma2d(st + p.x_atom, &pr.tm_x, chunk * kChunk + kAtom, 0, L.full + 8 * s, pol_x);
+                tma2d(st + p.x_bytes, &pr.tm_raw, chunk * kChunk, tile * kRows, L.full + 8 * s, pol_w);
+                tma2d(st + p.x_bytes + kRawBytes, &pr.tm_code, chunk * (kChunk / 2), tile * kRows, L.full + 8 * s,
                       pol_w);
                 ++issued;
                 if (++s == S) {
@@ -544,10 +588,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             const uint32_t idesc = instr_desc(p.Mp);
             int s = 0, a = 0;
             uint32_t round = 0, around = 0, tiles = 0;
-            int chunk = static_cast<int>(u0 % p.n_chunks);
-            for (long long u = u0; u < u1; ++u, chunk = (chunk + 1 == p.n_chunks) ? 0 : chunk + 1) {
-                const bool first = (u == u0) || chunk == 0;
-                const bool last = (u + 1 == u1) || chunk == p.n_chunks - 1;
+            UPos q = q0;
+            for (long long u = u0; u < u1; ++u, next(q, p)) {
+                const bool first = (u == u0) || q.chunk == 0;
+                const bool last = (u + 1 == u1) || q.chunk == p.prob[q.p].n_chunks - 1;
                 bool w = bar_wait(L.full + 8 * s, round & 1u) && bar_wait(L.a_full + 8 * a, around & 1u);
                 if (w && first) w = bar_wait(L.acc_empty, (tiles & 1u) ^ 1u);
                 if (!w) {
@@ -584,29 +628,30 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         // ---- decode warps (and the epilogue)
         const int ew = warp - 2;
         const int t = ew * 32 + lane;
-        const int q4 = t & 3, r = t >> 2;  // row r of each chunk, columns 16*q4 .. +15
+        const int q4 = t & 3, r = t >> 2;  // row r of each unit, columns 32*q4 .. +31
         int s = 0, a = 0;
         uint32_t round = 0, around = 0, tiles = 0;
         // the row metadata of the next two units is in flight while a unit is decoded
-        RowMeta m0 = {0, 0, 0, 0, 0}, m1 = {0, 0, 0, 0, 0};
-        UPos q = {static_cast<int>(u0 / p.n_chunks), static_cast<int>(u0 % p.n_chunks)};
+        RowMeta m0 = {0, 0, 0, 0, 0, 0}, m1 = {0, 0, 0, 0, 0, 0};
+        UPos q = q0;
         UPos qm = q;  // the unit whose metadata is loaded next
         if (u0 < u1) {
             m0 = load_row_meta(p, qm, r);
-            fetch_escapes(p, m0);
+            fetch_escapes(p.prob[m0.pi], m0);
         }
-        next(qm, p.n_chunks);
+        next(qm, p);
         if (u0 + 1 < u1) m1 = load_row_meta(p, qm, r);
-        next(qm, p.n_chunks);
-        for (long long u = u0; u < u1; ++u, next(q, p.n_chunks)) {
+        next(qm, p);
+        for (long long u = u0; u < u1; ++u, next(q, p)) {
+            const Problem &pr = p.prob[q.p];
             const int tile = q.tile, chunk = q.chunk;
-            const bool last = (u + 1 == u1) || chunk == p.n_chunks - 1;
+            const bool last = (u + 1 == u1) || chunk == pr.n_chunks - 1;
             RowMeta m2 = m1;
             if (u + 2 < u1) {
                 m2 = load_row_meta(p, qm, r);
-                next(qm, p.n_chunks);
+                next(qm, p);
             }
-            if (u + 1 < u1) fetch_escapes(p, m1);  // m1's offsets arrived during the previous unit
+            if (u + 1 < u1) fetch_escapes(p.prob[m1.pi], m1);  // m1's offsets arrived during the previous unit
             const bool w = bar_wait(L.full + 8 * s, round & 1u) && bar_wait(L.a_empty + 8 * a, (around & 1u) ^ 1u);
             if (!__all_sync(0xFFFFFFFFu, w)) {
                 raise_flag(p.err, S12_FLAG_TIMEOUT);
@@ -614,7 +659,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             }
             const uint32_t st = L.stages + static_cast<uint32_t>(s) * p.stage_bytes;
             const uint32_t aa = L.abuf + static_cast<uint32_t>(a) * kABytes;
-            decode_row<CHECK>(p, st + p.x_bytes, st + p.x_bytes + kRawBytes, aa, r, q4, m0);
+            decode_row<CHECK>(pr, p.err, st + p.x_bytes, st + p.x_bytes + kRawBytes, aa, r, q4, m0);
             m0 = m1;
             m1 = m2;
             // generic-proxy stores must be visible to the tensor core
@@ -640,7 +685,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                 }
                 ++tiles;
                 tc_fence_after();
-                epilogue(p, tmem, L, tile, u0, u1, ew, lane);
+                const long long t0 = pr.unit0 + static_cast<long long>(tile) * pr.n_chunks;
+                epilogue(p, pr, tmem, L, tile, pr.tile0 + tile, t0, u0, u1, ew, lane);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) bar_arrive(L.acc_empty);
@@ -664,19 +710,27 @@ namespace {
 constexpr uint32_t kSmemLimit = 227 * 1024;
 
 struct Plan {
-    int Mp, n_tiles, n_chunks, grid, stages;
+    int Mp, n_tiles, grid, stages;
     long long n_units;
     uint32_t x_bytes, x_atom, stage_bytes, tmem_cols, smem;
     int a_bufs;
     size_t part_bytes, cnt_bytes;
 };
 
-Plan plan(const s12_view *v, int M, int sms) {
+// One plan for `count` matrices with token rows M[i]; they share Mp, the
+// largest M rounded up to 16.
+Plan plan(const s12_view *views, int count, const int *M, int sms) {
     Plan pl;
-    pl.Mp = (M + 15) / 16 * 16;
-    pl.n_tiles = static_cast<int>((v->rows + gemm::kRows - 1) / gemm::kRows);
-    pl.n_chunks = static_cast<int>(v->cols / gemm::kChunk);
-    pl.n_units = static_cast<long long>(pl.n_tiles) * pl.n_chunks;
+    int mmax = 0;
+    pl.n_tiles = 0;
+    pl.n_units = 0;
+    for (int i = 0; i < count; ++i) {
+        mmax = std::max(mmax, M[i]);
+        const int tiles = static_cast<int>((views[i].rows + gemm::kRows - 1) / gemm::kRows);
+        pl.n_tiles += tiles;
+        pl.n_units += static_cast<long long>(tiles) * static_cast<long long>(views[i].cols / gemm::kChunk);
+    }
+    pl.Mp = (mmax + 15) / 16 * 16;
     pl.grid = static_cast<int>(std::max(1LL, std::min<long long>(sms, pl.n_units)));
     pl.x_atom = static_cast<uint32_t>(pl.Mp) * 128u;
     pl.x_bytes = 2 * pl.x_atom;
@@ -693,52 +747,50 @@ Plan plan(const s12_view *v, int M, int sms) {
     uint32_t cols = 32;
     while (cols < static_cast<uint32_t>(pl.Mp)) cols <<= 1;
     pl.tmem_cols = cols;
-    // sized for the largest grid so one workspace fits every call with this M
+    // sized for the largest grid so one workspace fits every call with this Mp
     pl.part_bytes = align_up(static_cast<uint64_t>(sms) * 2 * pl.Mp * gemm::kRows * sizeof(float), kAlign);
     pl.cnt_bytes = align_up(static_cast<uint64_t>(pl.n_tiles) * sizeof(uint32_t), kAlign);
     return pl;
 }
 
-}  // namespace
-
-size_t gemm_ws_bytes(const s12_view *v, int M) {
-    int sms = 0;
-    if (device_sms(&sms) != cudaSuccess) return 0;
-    const Plan pl = plan(v, M, sms);
-    return pl.part_bytes + pl.cnt_bytes;
-}
-
-int launch_gemm(const s12_view *v, const uint16_t *x, int M, float *y, void *ws, size_t ws_bytes, uint32_t *err,
-                cudaStream_t stream) {
-    int sms = 0;
-    if (device_sms(&sms) != cudaSuccess) return S12_ERR_CUDA;
-    const Plan pl = plan(v, M, sms);
-    if (!ws || ws_bytes < pl.part_bytes + pl.cnt_bytes) return S12_ERR_CAPACITY;
-    if (pl.stages < 2) return S12_ERR_SHAPE;
-    gemm::Params p = {};
-    const uint64_t N = v->rows, K = v->cols;
-    if (make_tmap_u8_2d(&p.tm_raw, v->raw, K, N, K, gemm::kChunk, gemm::kRows, true) != S12_OK) return S12_ERR_CUDA;
-    if (make_tmap_u8_2d(&p.tm_code, v->code, K / 2, N, K / 2, gemm::kChunk / 2, gemm::kRows, false) != S12_OK)
-        return S12_ERR_CUDA;
-    if (make_tmap_bf16_2d(&p.tm_x, x, K, static_cast<uint64_t>(M), K * 2, gemm::kAtom, static_cast<uint32_t>(pl.Mp),
-                          true) != S12_OK)
-        return S12_ERR_CUDA;
-    p.base = v->base;
-    p.esc_off = v->esc_off;
-    p.esc = v->esc;
-    p.code = v->code;
-    p.n_esc = v->n_esc;
-    p.y = y;
+template <bool CHECK, int NP>
+int run_gemm(const s12_view *views, int count, const uint16_t *const *x, const int *M, float *const *y, void *ws,
+             uint32_t *err, const Plan &pl, cudaStream_t stream) {
+    gemm::Params<NP> p = {};
+    long long unit0 = 0;
+    int tile0 = 0;
+    for (int i = 0; i < count; ++i) {
+        const s12_view *v = views + i;
+        gemm::Problem &q = p.prob[i];
+        const uint64_t N = v->rows, K = v->cols;
+        if (make_tmap_u8_2d(&q.tm_raw, v->raw, K, N, K, gemm::kChunk, gemm::kRows, true) != S12_OK)
+            return S12_ERR_CUDA;
+        if (make_tmap_u8_2d(&q.tm_code, v->code, K / 2, N, K / 2, gemm::kChunk / 2, gemm::kRows, false) != S12_OK)
+            return S12_ERR_CUDA;
+        if (make_tmap_bf16_2d(&q.tm_x, x[i], K, static_cast<uint64_t>(M[i]), K * 2, gemm::kAtom,
+                              static_cast<uint32_t>(pl.Mp), true) != S12_OK)
+            return S12_ERR_CUDA;
+        q.base = v->base;
+        q.esc_off = v->esc_off;
+        q.esc = v->esc;
+        q.n_esc = v->n_esc;
+        q.y = y[i];
+        q.N = static_cast<int>(N);
+        q.K = static_cast<int>(K);
+        q.T = q.K / kTile;
+        q.M = M[i];
+        q.n_tiles = static_cast<int>((N + gemm::kRows - 1) / gemm::kRows);
+        q.n_chunks = static_cast<int>(K / gemm::kChunk);
+        q.unit0 = unit0;
+        q.tile0 = tile0;
+        unit0 += static_cast<long long>(q.n_tiles) * q.n_chunks;
+        tile0 += q.n_tiles;
+    }
     p.part = static_cast<float *>(ws);
     p.cnt = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(ws) + pl.part_bytes);
     p.err = err;
-    p.N = static_cast<int>(N);
-    p.K = static_cast<int>(K);
-    p.T = p.K / kTile;
-    p.M = M;
+    p.n_problems = count;
     p.Mp = pl.Mp;
-    p.n_tiles = pl.n_tiles;
-    p.n_chunks = pl.n_chunks;
     p.n_units = pl.n_units;
     p.stages = pl.stages;
     p.stage_bytes = pl.stage_bytes;
@@ -746,11 +798,35 @@ int launch_gemm(const s12_view *v, const uint16_t *x, int M, float *y, void *ws,
     p.x_atom = pl.x_atom;
     p.a_bufs = pl.a_bufs;
     p.tmem_cols = pl.tmem_cols;
-    auto kern = err ? gemm::gemm_tc_kernel<true> : gemm::gemm_tc_kernel<false>;
+    auto kern = gemm::gemm_tc_kernel<CHECK, NP>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem) != cudaSuccess)
         return S12_ERR_CUDA;
     kern<<<pl.grid, gemm::kThreads, pl.smem, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? S12_OK : S12_ERR_CUDA;
+}
+
+}  // namespace
+
+size_t gemm_ws_bytes(const s12_view *views, int count, const int *M) {
+    int sms = 0;
+    if (device_sms(&sms) != cudaSuccess) return 0;
+    const Plan pl = plan(views, count, M, sms);
+    return pl.part_bytes + pl.cnt_bytes;
+}
+
+int launch_gemm(const s12_view *views, int count, const uint16_t *const *x, const int *M, float *const *y, void *ws,
+                size_t ws_bytes, uint32_t *err, cudaStream_t stream) {
+    int sms = 0;
+    if (device_sms(&sms) != cudaSuccess) return S12_ERR_CUDA;
+    const Plan pl = plan(views, count, M, sms);
+    if (!ws || ws_bytes < pl.part_bytes + pl.cnt_bytes) return S12_ERR_CAPACITY;
+    if (pl.stages < 2) return S12_ERR_SHAPE;
+    // a one-matrix call takes the small parameter block
+    if (count == 1)
+        return err ? run_gemm<true, 1>(views, count, x, M, y, ws, err, pl, stream)
+                   : run_gemm<false, 1>(views, count, x, M, y, ws, err, pl, stream);
+    return err ? run_gemm<true, gemm::kMaxProblems>(views, count, x, M, y, ws, err, pl, stream)
+               : run_gemm<false, gemm::kMaxProblems>(views, count, x, M, y, ws, err, pl, stream);
 }
 
 }  // namespace s12

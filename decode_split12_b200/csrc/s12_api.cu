@@ -216,20 +216,55 @@ int s12_gemv(const s12_view *v, const uint16_t *x, int B, float *y, void *ws, si
 
 size_t s12_gemm_ws_bytes(const s12_view *v, int M) {
     if (check_view(v) != S12_OK || M < S12_GEMM_MIN_M || M > S12_GEMM_MAX_M) return 0;
-    return gemm_ws_bytes(v, M);
+    return gemm_ws_bytes(v, 1, &M);
 }
+
+namespace {
+// Shared checks of the GEMM calls: every entry valid, before any launch.
+// min_m: the smallest token count an entry may have (a grouped call pads
+// every matrix to the shared multiple of 16, so it accepts any M >= 1).
+int check_gemm_group(const s12_view *views, int count, const uint16_t *const *x, const int *M, float *const *y,
+                     int min_m) {
+    if (!views || !x || !M || !y || count < 1 || count > S12_GEMM_MAX_PROBLEMS) return S12_ERR_ARG;
+    for (int i = 0; i < count; ++i) {
+        const int rc = check_view(views + i);
+        if (rc != S12_OK) return rc;
+        if (!x[i] || !y[i]) return S12_ERR_ARG;
+        if (M[i] < min_m || M[i] > S12_GEMM_MAX_M) return S12_ERR_SHAPE;
+        if (views[i].rows > 0x7FFFFFFFull || views[i].cols > 0x7FFFFFFFull) return S12_ERR_SHAPE;
+        if (!aligned16(x[i]) || !aligned4(y[i])) return S12_ERR_ALIGN;
+    }
+    return S12_OK;
+}
+}  // namespace
 
 int s12_gemm_skinny(const s12_view *v, const uint16_t *x, int M, float *y, void *ws, size_t ws_bytes,
                     uint32_t *err_flag, void *stream) {
     int rc = check_view(v);
     if (rc != S12_OK) return rc;
     if (!x || !y) return S12_ERR_ARG;
-    if (M < S12_GEMM_MIN_M || M > S12_GEMM_MAX_M) return S12_ERR_SHAPE;
-    if (v->rows > 0x7FFFFFFFull || v->cols > 0x7FFFFFFFull) return S12_ERR_SHAPE;
-    if (!aligned16(x) || !aligned4(y) || (ws && !aligned16(ws)) || (err_flag && !aligned4(err_flag)))
-        return S12_ERR_ALIGN;
-    if (ws_bytes < gemm_ws_bytes(v, M)) return S12_ERR_CAPACITY;
-    return launch_gemm(v, x, M, y, ws, ws_bytes, err_flag, static_cast<cudaStream_t>(stream));
+    rc = check_gemm_group(v, 1, &x, &M, &y, S12_GEMM_MIN_M);
+    if (rc != S12_OK) return rc;
+    if ((ws && !aligned16(ws)) || (err_flag && !aligned4(err_flag))) return S12_ERR_ALIGN;
+    if (ws_bytes < gemm_ws_bytes(v, 1, &M)) return S12_ERR_CAPACITY;
+    return launch_gemm(v, 1, &x, &M, &y, ws, ws_bytes, err_flag, static_cast<cudaStream_t>(stream));
+}
+
+size_t s12_gemm_multi_ws_bytes(const s12_view *views, int count, const int *M) {
+    if (!views || !M || count < 1 || count > S12_GEMM_MAX_PROBLEMS) return 0;
+    for (int i = 0; i < count; ++i)
+        if (check_view(views + i) != S12_OK || M[i] < 1 || M[i] > S12_GEMM_MAX_M) return 0;
+    return gemm_ws_bytes(views, count, M);
+}
+
+int s12_gemm_skinny_multi(const s12_view *views, int count, const uint16_t *const *x, const int *M,
+                          float *const *y, void *ws, size_t ws_bytes, uint32_t *err_flag, void *stream) {
+    const int rc = check_gemm_group(views, count, x, M, y, 1);
+    if (rc != S12_OK) return rc;
+    if (!ws) return S12_ERR_ARG;
+    if (!aligned16(ws) || (err_flag && !aligned4(err_flag))) return S12_ERR_ALIGN;
+    if (ws_bytes < gemm_ws_bytes(views, count, M)) return S12_ERR_CAPACITY;
+    return launch_gemm(views, count, x, M, y, ws, ws_bytes, err_flag, static_cast<cudaStream_t>(stream));
 }
 
 size_t s12_stats_ws_bytes(void) { return 256 * sizeof(unsigned long long); }

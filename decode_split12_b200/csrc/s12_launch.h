@@ -32,8 +32,8 @@ size_t encode_ws_bytes(int64_t rows, int64_t cols);
 int launch_encode(const uint16_t *w, int64_t rows, int64_t cols, void *dst, size_t dst_cap, size_t *bytes_out,
                   void *ws, size_t ws_bytes, cudaStream_t stream);
 int launch_stats_hist(const s12_view *v, unsigned long long *hist_dev, cudaStream_t stream);
-size_t gemm_ws_bytes(const s12_view *v, int M);
-int launch_gemm(const s12_view *v, const uint16_t *x, int M, float *y, void *ws, size_t ws_bytes, uint32_t *err,
-                cudaStream_t stream);
+size_t gemm_ws_bytes(const s12_view *views, int count, const int *M);
+int launch_gemm(const s12_view *views, int count, const uint16_t *const *x, const int *M, float *const *y, void *ws,
+                size_t ws_bytes, uint32_t *err, cudaStream_t stream);
 
 }  // namespace s12

@@ -35,7 +35,8 @@ S12_FLAG_TIMEOUT = 8
 EXPORTED = (
     "s12_error_string", "s12_device_check", "s12_container_bytes", "s12_encode_ws_bytes", "s12_encode",
     "s12_open", "s12_decode", "s12_gemv_ws_bytes", "s12_gemv", "s12_gemv_multi_ws_bytes", "s12_gemv_multi",
-    "s12_gemv_noalloc", "s12_gemm_ws_bytes", "s12_gemm_skinny", "s12_stats_ws_bytes",
+    "s12_gemv_noalloc", "s12_gemm_ws_bytes", "s12_gemm_skinny", "s12_gemm_multi_ws_bytes",
+    "s12_gemm_skinny_multi", "s12_stats_ws_bytes",
     "s12_stats", "s12_bf16_gemv",
 )
 
@@ -106,6 +107,11 @@ def _lib() -> C.CDLL:
         lib.s12_gemm_ws_bytes.restype = _SZ
         lib.s12_gemm_skinny.argtypes = [C.POINTER(View), _P, C.c_int, _P, _P, _SZ, _P, _P]
         lib.s12_gemm_skinny.restype = C.c_int
+        lib.s12_gemm_multi_ws_bytes.argtypes = [C.POINTER(View), C.c_int, C.POINTER(C.c_int)]
+        lib.s12_gemm_multi_ws_bytes.restype = _SZ
+        lib.s12_gemm_skinny_multi.argtypes = [C.POINTER(View), C.c_int, C.POINTER(_P), C.POINTER(C.c_int),
+                                              C.POINTER(_P), _P, _SZ, _P, _P]
+        lib.s12_gemm_skinny_multi.restype = C.c_int
         lib.s12_stats_ws_bytes.argtypes = []
         lib.s12_stats_ws_bytes.restype = _SZ
         lib.s12_stats.argtypes = [C.POINTER(View), C.POINTER(Stats), _P, _SZ, _P]
@@ -320,3 +326,29 @@ def s12_bf16_gemv(w: torch.Tensor, x: torch.Tensor, y: torch.Tensor | None = Non
         y = torch.empty((B, rows), dtype=torch.float32, device=x.device)
     _check(_lib().s12_bf16_gemv(_dptr(w), rows, cols, _dptr(x), B, _dptr(y), _stream(stream)), "s12_bf16_gemv")
     return y
+
+
+def s12_gemm_multi_ws_bytes(views, Ms) -> int:
+    ma = (C.c_int * len(Ms))(*[int(m) for m in Ms])
+    return int(_lib().s12_gemm_multi_ws_bytes(_view_array(views), len(views), ma))
+
+
+def s12_gemm_skinny_multi(views, xs, ys=None, ws: torch.Tensor | None = None, err_flag: torch.Tensor | None = None,
+                          stream=None):
+    """Several independent fused decode-skinny-GEMMs in one launch (each x_i
+    is M_i x cols_i); returns the list of y tensors (allocated when `ys` is
+    None)."""
+    xs = [_u16(x) for x in xs]
+    Ms = [int(x.shape[0]) for x in xs]
+    if ys is None:
+        ys = [torch.empty((m, v.rows), dtype=torch.float32, device=xs[0].device) for m, v in zip(Ms, views)]
+    arr = _view_array(views)
+    ma = (C.c_int * len(Ms))(*Ms)
+    if ws is None:
+        need = max(int(_lib().s12_gemm_multi_ws_bytes(arr, len(views), ma)), 256)
+        ws = torch.zeros(need, dtype=torch.uint8, device=xs[0].device)
+    xp = (_P * len(xs))(*[_dptr(x) for x in xs])
+    yp = (_P * len(ys))(*[_dptr(y) for y in ys])
+    _check(_lib().s12_gemm_skinny_multi(arr, len(views), xp, ma, yp, _dptr(ws), ws.numel(), _dptr(err_flag),
+                                        _stream(stream)), "s12_gemm_skinny_multi")
+    return ys

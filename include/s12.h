@@ -83,6 +83,7 @@ extern "C" {
 #define S12_GEMV_MAX_PROBLEMS 8 /* matrices in one s12_gemv_multi call */
 #define S12_GEMM_MIN_M 16
 #define S12_GEMM_MAX_M 256
+#define S12_GEMM_MAX_PROBLEMS 16 /* matrices per s12_gemm_skinny_multi call */
 
 /* Host-side description of an opened container.  All pointers are device
  * pointers into the caller's container buffer. */
@@ -241,11 +242,39 @@ size_t s12_gemm_ws_bytes(const s12_view *v, int M);
 
 /* y[m][n] = sum_k W[n][k] * x[m][k] for 16 <= M <= 256.
  *   x: device BF16, M x cols row-major.  y: device FP32, M x rows row-major,
- *   overwritten.  ws: device scratch of s12_gemm_ws_bytes(v, M) bytes.
+ *   overwritten.  ws: device scratch of s12_gemm_ws_bytes(v, M) bytes,
+ *   ZERO-FILLED before its first use; every call leaves it zero-filled.
  * Decoded BF16 tiles are written to shared memory and multiplied by the
  * tensor cores with FP32 accumulation. */
 int s12_gemm_skinny(const s12_view *v, const uint16_t *x, int M, float *y, void *ws,
                     size_t ws_bytes, uint32_t *err_flag, void *stream);
+
+/* Workspace bytes s12_gemm_skinny_multi needs for these `count` containers
+ * with token rows M[i] (0 for invalid arguments). */
+size_t s12_gemm_multi_ws_bytes(const s12_view *views, int count, const int *M);
+
+/* Up to S12_GEMM_MAX_PROBLEMS independent fused decode-skinny-GEMMs in ONE
+ * kernel launch: for i < count, y[i][m][n] = sum_k W_i[n][k] * x[i][m][k]
+ * for m < M[i], 1 <= M[i] <= 256 (below 16 too: every matrix is multiplied
+ * at the call's shared padded M).  Built for a mixture-of-experts block,
+ * where each expert's matrices see a different number of routed tokens.
+ *   views: host array of `count` opened containers (shapes may differ).
+ *   x, y:  host arrays of `count` device pointers, laid out as in
+ *          s12_gemm_skinny (x[i]: M[i] x cols_i bf16, y[i]: M[i] x rows_i
+ *          fp32, overwritten).
+ *   M:     host array of the token rows of each matrix.
+ *   ws:    device workspace of s12_gemm_multi_ws_bytes bytes, zero-filled
+ *          before its first use and left zero-filled (as for
+ *          s12_gemm_skinny).
+ * The 128-row x 128-column units of all matrices are dealt to the SMs as one
+ * range, so the launch, ramp-up and tail are paid once for the group.  All
+ * matrices are multiplied at the largest M rounded up to 16 (rows of x past
+ * a matrix's own M are read as zeros and never stored), so matrices of
+ * similar M group best.  Each y[i] equals what s12_gemm_skinny gives for
+ * that matrix up to the summation order, within the same tolerance.  A bad
+ * entry fails the whole call before any launch. */
+int s12_gemm_skinny_multi(const s12_view *views, int count, const uint16_t *const *x, const int *M,
+                          float *const *y, void *ws, size_t ws_bytes, uint32_t *err_flag, void *stream);
 
 /* ---- statistics ([M] section 1: exponent entropy; [T] key points:
  * escape rate) ---- */

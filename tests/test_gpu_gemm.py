@@ -96,3 +96,85 @@ def test_gemm_70b_mlp_full_size_sampled(s12, oracle, name, M):
     rows = np.unique(np.concatenate([[0, w.shape[0] - 1], wl.rng_for(8, M).choice(w.shape[0], 46, replace=False)]))
     yr, sr = oracle.gemv_rows_f64(host, x, rows)
     assert_within_tolerance(y[:, rows], yr, sr)
+
+
+# ---------------------------------------------------------------------------
+# grouped launch (s12_gemm_skinny_multi)
+
+@pytest.mark.parametrize("checked", [True, False])
+def test_gemm_multi_mixed_shapes_and_tokens(s12, oracle, checked):
+    """Six matrices of different shapes (ragged 128-row tiles, long rows,
+    a matrix smaller than one tile) and different token counts (one below
+    16) in one launch:
+    every y_i matches the FP64 oracle, and the rows of the shared padded
+    token count beyond M_i are never written."""
+    shapes = [(300, 1152), (128, 128), (77, 4096), (640, 1024), (16, 2048), (200, 512)]
+    Ms = [17, 32, 16, 29, 24, 3]
+    ws_, xs, views, blobs = [], [], [], []
+    for i, ((r, c), m) in enumerate(zip(shapes, Ms)):
+        w = wl.normal_with_outliers(r, c, 0.02, 0.002, 40 + i)
+        ws_.append(w)
+        xs.append(wl.activations(m, c, 50 + i))
+        blobs.append(s12.s12_encode(to_dev(w)))
+        views.append(s12.s12_open(blobs[-1]))
+    ys = [torch.full((m, r), float("nan"), dtype=torch.float32, device="cuda") for m, (r, _) in zip(Ms, shapes)]
+    flag = new_flag() if checked else None
+    s12.s12_gemm_skinny_multi(views, [to_dev(x) for x in xs], ys, err_flag=flag)
+    torch.cuda.synchronize()
+    for w, x, y in zip(ws_, xs, ys):
+        yr, sr = oracle.gemv_f64(oracle.encode(w), x)
+        assert_within_tolerance(y.cpu().numpy(), yr, sr)
+    if checked:
+        assert int(flag.item()) == 0
+
+
+def test_gemm_multi_moe_experts_full_size(s12, oracle):
+    """An 8-expert block's gate projections (14336 x 4096 each) with the
+    token counts of a top-2 routing of 64 tokens, in one launch; 24 sampled
+    rows per expert against the FP64 oracle, and the result equals the
+    per-expert single calls within the tolerance."""
+    Ms = [14, 15, 13, 14, 17, 20, 15, 20]
+    views, blobs, hosts, xs = [], [], [], []
+    for e, m in enumerate(Ms):
+        w = wl.student_t_scaled(14336, 4096, 100 + e)
+        blobs.append(s12.s12_encode(to_dev(w)))
+        views.append(s12.s12_open(blobs[-1]))
+        hosts.append(blobs[-1].cpu().numpy())
+        xs.append(wl.activations(m, 4096, 200 + e))
+        del w
+    ys = s12.s12_gemm_skinny_multi(views, [to_dev(x) for x in xs])
+    torch.cuda.synchronize()
+    for e, m in enumerate(Ms):
+        rows = np.unique(np.concatenate([[0, 14335], wl.rng_for(9, e).choice(14336, 22, replace=False)]))
+        yr, sr = oracle.gemv_rows_f64(hosts[e], xs[e], rows)
+        assert_within_tolerance(ys[e][:, rows].cpu().numpy(), yr, sr)
+
+
+def test_gemm_multi_deterministic_and_workspace_clean(s12):
+    """Two identical grouped calls give identical outputs and leave the
+    workspace's arrival counters at zero."""
+    mats = [wl.student_t_scaled(1024, 4096, 3), wl.student_t_scaled(512, 2048, 4)]
+    views = [s12.s12_open(s12.s12_encode(to_dev(w))) for w in mats]
+    xs = [to_dev(wl.activations(48, 4096, 3)), to_dev(wl.activations(40, 2048, 4))]
+    need = s12.s12_gemm_multi_ws_bytes(views, [48, 40])
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    a = s12.s12_gemm_skinny_multi(views, xs, ws=ws)
+    b = s12.s12_gemm_skinny_multi(views, xs, ws=ws)
+    torch.cuda.synchronize()
+    for ya, yb in zip(a, b):
+        assert torch.equal(ya, yb)
+    n_tiles = (1024 + 127) // 128 + (512 + 127) // 128
+    n_cnt = -(-n_tiles * 4 // 256) * 256
+    assert int(ws[-n_cnt:].count_nonzero()) == 0
+
+
+def test_gemm_multi_rejects_bad_groups(s12):
+    """More than S12_GEMM_MAX_PROBLEMS matrices, or an M above 256 in any
+    entry, fails the whole call before any launch."""
+    w = wl.normal_with_outliers(128, 256, 0.02, 0.0, 1)
+    v = s12.s12_open(s12.s12_encode(to_dev(w)))
+    x = to_dev(wl.activations(16, 256, 0))
+    with pytest.raises(s12.S12Error):
+        s12.s12_gemm_skinny_multi([v] * 17, [x] * 17)
+    with pytest.raises(s12.S12Error):
+        s12.s12_gemm_skinny_multi([v, v], [x, to_dev(wl.activations(257, 256, 0))])
