@@ -55,7 +55,7 @@ constexpr uint32_t kRawBytes = kRows * kChunk;       // 16 KB
 constexpr uint32_t kCodeBytes = kRows * kChunk / 2;  // 8 KB
 constexpr uint32_t kAtomBytes = kRows * kAtom * 2;   // 16 KB: one swizzle atom of the decoded unit
 constexpr uint32_t kABytes = 2 * kAtomBytes;         // 32 KB
-constexpr int kMaxABufs = 2;
+constexpr int kMaxABufs = 3;
 constexpr int kMaxStages = 6;
 constexpr int kMaxProblems = S12_GEMM_MAX_PROBLEMS;
 
@@ -370,7 +370,7 @@ __device__ __forceinline__ void decode_row(const Problem &p, uint32_t *err, uint
     const uint32_t lo = rm.lo, hi = rm.hi;
     const uint4 rw0 = lds128(st_raw + r * 128 + (((2u * q4) ^ sw) << 4));  // raw rows are 128-byte swizzled
     const uint4 rw1 = lds128(st_raw + r * 128 + (((2u * q4 + 1u) ^ sw) << 4));
-    uint4 code = lds128(st_code + r * 64 + 16 * q4);
+    uint4 code = lds128(st_code + r * 64 + 16 * (static_cast<uint32_t>(q4) ^ ((static_cast<uint32_t>(r) >> 1) & 3u)));
     bool esc = lo != hi;
     uint2 m0 = make_uint2(0, 0), m1 = make_uint2(0, 0);
     if (CHECK) {
@@ -393,10 +393,10 @@ __device__ __forceinline__ void decode_row(const Problem &p, uint32_t *err, uint
         uint32_t incl = n;
 #pragma unroll
         for (int d = 1; d < 4; d <<= 1) {
-            const uint32_t v = __shfl_up_sync(quads, incl, d, 4);
+            const uint32_t v = __shfl_up_sync(quads, incl, 8 * d);
             if (q4 >= d) incl += v;
         }
-        const uint32_t tot = __shfl_sync(quads, incl, 3, 4);
+        const uint32_t tot = __shfl_sync(quads, incl, 24 + (r & 7));
         if (q4 == 0 && tot != hi - lo) raise_flag(err, S12_FLAG_ESC_COUNT);
         s0 = lo + incl - n;
         s1 = s0 + n0;
@@ -627,8 +627,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     } else {
         // ---- decode warps (and the epilogue)
         const int ew = warp - 2;
-        const int t = ew * 32 + lane;
-        const int q4 = t & 3, r = t >> 2;  // row r of each unit, columns 32*q4 .. +31
+        const int q4 = lane >> 3, r = 8 * ew + (lane & 7);  // row r of each unit, columns 32*q4 .. +31
         int s = 0, a = 0;
         uint32_t round = 0, around = 0, tiles = 0;
         // the row metadata of the next two units is in flight while a unit is decoded
@@ -735,13 +734,13 @@ Plan plan(const s12_view *views, int count, const int *M, int sms) {
     pl.x_atom = static_cast<uint32_t>(pl.Mp) * 128u;
     pl.x_bytes = 2 * pl.x_atom;
     pl.stage_bytes = pl.x_bytes + gemm::kRawBytes + gemm::kCodeBytes;
-    // two decoded-unit buffers when two stages still fit beside them, else one
+    // three decoded-unit buffers when three stages still fit beside them, else fewer
     pl.a_bufs = gemm::kMaxABufs;
     uint32_t fixed = 0;
     for (;; --pl.a_bufs) {
         fixed = 1024 + 1024 + static_cast<uint32_t>(pl.a_bufs) * gemm::kABytes;  // slack, barriers, A buffers
         pl.stages = static_cast<int>(std::min<uint32_t>(gemm::kMaxStages, (kSmemLimit - fixed) / pl.stage_bytes));
-        if (pl.stages >= 2 || pl.a_bufs == 1) break;
+        if (pl.stages >= (pl.a_bufs == 3 ? 3 : 2) || pl.a_bufs == 1) break;
     }
     pl.smem = fixed + static_cast<uint32_t>(pl.stages) * pl.stage_bytes;
     uint32_t cols = 32;
@@ -763,12 +762,12 @@ int run_gemm(const s12_view *views, int count, const uint16_t *const *x, const i
         const s12_view *v = views + i;
         gemm::Problem &q = p.prob[i];
         const uint64_t N = v->rows, K = v->cols;
-        if (make_tmap_u8_2d(&q.tm_raw, v->raw, K, N, K, gemm::kChunk, gemm::kRows, true) != S12_OK)
+        if (make_tmap_u8_2d(&q.tm_raw, v->raw, K, N, K, gemm::kChunk, gemm::kRows, 128) != S12_OK)
             return S12_ERR_CUDA;
-        if (make_tmap_u8_2d(&q.tm_code, v->code, K / 2, N, K / 2, gemm::kChunk / 2, gemm::kRows, false) != S12_OK)
+        if (make_tmap_u8_2d(&q.tm_code, v->code, K / 2, N, K / 2, gemm::kChunk / 2, gemm::kRows, 64) != S12_OK)
             return S12_ERR_CUDA;
         if (make_tmap_bf16_2d(&q.tm_x, x[i], K, static_cast<uint64_t>(M[i]), K * 2, gemm::kAtom,
-                              static_cast<uint32_t>(pl.Mp), true) != S12_OK)
+                              static_cast<uint32_t>(pl.Mp), 128) != S12_OK)
             return S12_ERR_CUDA;
         q.base = v->base;
         q.esc_off = v->esc_off;

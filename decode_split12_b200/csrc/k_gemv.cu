@@ -592,9 +592,9 @@ int run(const s12_view *views, int count, const uint16_t *const *x, int B, float
         const s12_view *v = views + i;
         gemv::Problem &m = pr.prob[i];
         const uint64_t R = v->rows, K = v->cols;
-        if (make_tmap_u8_2d(&m.tm_raw, v->raw, K, R, K, 128, gemv::kRowsPerGroup, true) != S12_OK)
+        if (make_tmap_u8_2d(&m.tm_raw, v->raw, K, R, K, 128, gemv::kRowsPerGroup, 128) != S12_OK)
             return S12_ERR_CUDA;
-        if (make_tmap_u8_2d(&m.tm_code, v->code, K / 2, R, K / 2, 64, gemv::kRowsPerGroup, false) != S12_OK)
+        if (make_tmap_u8_2d(&m.tm_code, v->code, K / 2, R, K / 2, 64, gemv::kRowsPerGroup, 0) != S12_OK)
             return S12_ERR_CUDA;
         m.base = v->base;
         m.esc_off = v->esc_off;

@@ -58,24 +58,24 @@ std::once_flag g_encode_once;
 
 namespace {
 int encode_2d(CUtensorMap *out, CUtensorMapDataType dtype, const void *base, uint64_t inner, uint64_t rows,
-              uint64_t row_stride, uint32_t box_inner, uint32_t box_rows, bool swizzle128);
+              uint64_t row_stride, uint32_t box_inner, uint32_t box_rows, int swizzle);
 }  // namespace
 
 int make_tmap_bf16_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t rows, uint64_t row_stride,
-                      uint32_t box_inner, uint32_t box_rows, bool swizzle128) {
+                      uint32_t box_inner, uint32_t box_rows, int swizzle) {
     return encode_2d(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, inner, rows, row_stride, box_inner, box_rows,
-                     swizzle128);
+                     swizzle);
 }
 
 int make_tmap_u8_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t rows, uint64_t row_stride,
-                    uint32_t box_inner, uint32_t box_rows, bool swizzle128) {
+                    uint32_t box_inner, uint32_t box_rows, int swizzle) {
     return encode_2d(out, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, inner, rows, row_stride, box_inner, box_rows,
-                     swizzle128);
+                     swizzle);
 }
 
 namespace {
 int encode_2d(CUtensorMap *out, CUtensorMapDataType dtype, const void *base, uint64_t inner, uint64_t rows,
-              uint64_t row_stride, uint32_t box_inner, uint32_t box_rows, bool swizzle128) {
+              uint64_t row_stride, uint32_t box_inner, uint32_t box_rows, int swizzle) {
     std::call_once(g_encode_once, [] {
         void *fn = nullptr;
         cudaDriverEntryPointQueryResult q;
@@ -90,7 +90,9 @@ int encode_2d(CUtensorMap *out, CUtensorMapDataType dtype, const void *base, uin
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = g_encode_tiled(out, dtype, 2, const_cast<void *>(base), dims, strides, box,
                                 estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                                swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                                swizzle == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : swizzle == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                : CU_TENSOR_MAP_SWIZZLE_NONE,
                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? S12_OK : S12_ERR_CUDA;
 }

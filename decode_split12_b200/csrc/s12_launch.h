@@ -13,14 +13,15 @@ cudaError_t device_sms(int *sms);
 
 // Tiled TMA descriptor for a row-major 2-D array of bytes: `inner` bytes
 // per row, `rows` rows, `row_stride` bytes between rows (multiple of 16),
-// box of box_inner x box_rows bytes (box_inner a multiple of 16; 128 with
-// the 128-byte swizzle), out-of-bounds bytes read as 0.
+// box of box_inner x box_rows bytes (box_inner a multiple of 16, and at most
+// the swizzle width), out-of-bounds bytes read as 0.  swizzle: 0 (none), 64
+// or 128 (the copy engine's 64- or 128-byte swizzle of 16-byte chunks).
 int make_tmap_u8_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t rows, uint64_t row_stride,
-                    uint32_t box_inner, uint32_t box_rows, bool swizzle128);
+                    uint32_t box_inner, uint32_t box_rows, int swizzle);
 // The same for a row-major 2-D array of BF16 values (`inner` and the box's
 // inner extent counted in elements, `row_stride` in bytes).
 int make_tmap_bf16_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t rows, uint64_t row_stride,
-                      uint32_t box_inner, uint32_t box_rows, bool swizzle128);
+                      uint32_t box_inner, uint32_t box_rows, int swizzle);
 
 int launch_decode(const s12_view *v, uint16_t *out, uint32_t *err, cudaStream_t stream);
 size_t gemv_ws_bytes(const s12_view *views, int count);
