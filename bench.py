@@ -438,6 +438,8 @@ def run_llama8b(args, world, rank):
         extra[name] = {"us_per_layer": round(sb * 1e6, 2), "GBs": round(2 * layer.weights / sb / 1e9, 1),
                        "hbm_frac": round(2 * layer.weights / sb / 1e9 / hbm, 4)}
         del gb
+    if layer.w_dev:
+        extra["mlp_swiglu_epilogue"] = mlp_swiglu_extras(layer, world, max(20, args.steps // 4))
     e2e_t, h2d, d2h, ge = e2e_llama(layer, max(20, args.steps // 2), args.warmup, world)
     if not args.no_gemm:
         del layer.w_dev
@@ -582,6 +584,50 @@ def _student_t_gpu(rows: int, cols: int, gen):
     t = z / torch.sqrt(2.0 * gam / 5.0)
     del z, gam
     return (t * (1.0 / math.sqrt(5.0 / 3.0) / math.sqrt(cols))).to(torch.bfloat16).view(torch.int16)
+
+
+def mlp_swiglu_extras(layer, world, steps: int):
+    """The layer's MLP at its batch: h = silu(gate x) * (up x), then down h.
+    Fused: one s12_gemv_swiglu over the interleaved gate/up container (h
+    written once, as BF16) and one s12_gemv for down.  Unfused: the gate and
+    up GEMVs in one grouped launch (FP32 outputs), torch's silu, multiply and
+    BF16 cast, then the down GEMV."""
+    import torch
+
+    from decode_split12_b200 import s12
+    hbm, _, _, _ = load_peaks()
+    B = layer.x["gate"].shape[0]
+    wi = s12.interleave_gate_up(layer.w_dev["gate"], layer.w_dev["up"])
+    blob = s12.s12_encode(wi)
+    del wi
+    gu = s12.s12_open(blob)
+    F = layer.views["gate"].rows
+    h = torch.empty((B, F), dtype=torch.int16, device="cuda")
+    yd = torch.empty((B, layer.views["down"].rows), dtype=torch.float32, device="cuda")
+    xg = layer.x["gate"]
+    yg = torch.empty((B, F), dtype=torch.float32, device="cuda")
+    yu = torch.empty((B, F), dtype=torch.float32, device="cuda")
+
+    def fused():
+        s12.s12_gemv_swiglu(gu, xg, h, ws=layer.ws)
+        s12.s12_gemv(layer.views["down"], h, yd, ws=layer.ws)
+
+    def unfused():
+        s12.s12_gemv_multi([layer.views["gate"], layer.views["up"]], [xg, xg], [yg, yu], ws=layer.ws)
+        hh = (torch.nn.functional.silu(yg) * yu).to(torch.bfloat16).view(torch.int16)
+        s12.s12_gemv(layer.views["down"], hh, yd, ws=layer.ws)
+
+    out = {"batch": B}
+    cbytes = int(gu.container_bytes) + int(layer.views["down"].container_bytes)
+    for name, fn in (("fused", fused), ("unfused", unfused)):
+        g = capture(fn)
+        for _ in range(3):
+            g.replay()
+        t = time_graph(g, steps, world) / steps
+        out[name] = {"us": round(t * 1e6, 2), "hbm_frac": round(cbytes / t / 1e9 / hbm, 4)}
+        del g
+    del blob, gu
+    return out
 
 
 def stack_extras(world, layers: int = 32, steps: int = 10):

@@ -46,6 +46,8 @@
 // for it.
 #include <algorithm>
 
+#include <cuda_bf16.h>
+
 #include "s12_device.cuh"
 #include "s12_launch.h"
 
@@ -73,11 +75,13 @@ struct __align__(64) Problem {
     const uint32_t *esc_off;
     const uint16_t *esc;
     const uint16_t *x;    // B x K bf16
-    float *y;             // B x R fp32
+    float *y;             // B x R fp32 (act = 0)
+    uint16_t *h;          // B x R/2 bf16 (act = 1)
     uint64_t n_esc;
     long long block0;     // first block of this matrix in the grouped numbering
     int R, K, T, n_groups;
     int group0;           // first row group of this matrix in the grouped numbering
+    int act;              // epilogue: 0 = y fp32; 1 = SwiGLU of interleaved gate/up rows into h
 };
 
 struct __align__(64) Params {
@@ -228,6 +232,24 @@ namespace gemv {
 // (g, q) holds D[g][2q], D[g][2q+1], D[g+8][2q], D[g+8][2q+1] (row of W,
 // batch row).
 __device__ __forceinline__ void store_y(const Problem &m, int B, const float (&a)[4], int grp, int g, int q) {
+    if (m.act) {
+        // SwiGLU epilogue.  The matrix interleaves the gate and up
+        // projections in blocks of 8 rows (rows 16i .. 16i+7 are gate rows
+        // 8i .. 8i+7, rows 16i+8 .. 16i+15 the up rows with the same
+        // indices), so this lane holds gate row f and up row f of the same
+        // batch columns: h[b][f] = silu(gate) * up, rounded to BF16.
+        const int f = grp * 8 + g, F = m.R >> 1;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int b = 2 * q + i;
+            if (f < F && b < B) {
+                const float gt = a[i], up = a[2 + i];
+                const float hv = gt / (1.f + expf(-gt)) * up;
+                m.h[static_cast<size_t>(b) * F + f] = __bfloat16_as_ushort(__float2bfloat16_rn(hv));
+            }
+        }
+        return;
+    }
     const int rA = grp * kRowsPerGroup + g;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -583,8 +605,8 @@ Plan plan(const s12_view *views, int count, int sms) {
 }
 
 template <bool CHECK>
-int run(const s12_view *views, int count, const uint16_t *const *x, int B, float *const *y, void *ws,
-        uint32_t *err, const Plan &pl, cudaStream_t stream) {
+int run(const s12_view *views, int count, const uint16_t *const *x, int B, void *const *y, const int *act,
+        void *ws, uint32_t *err, const Plan &pl, cudaStream_t stream) {
     gemv::Params pr = {};
     long long block0 = 0;
     int group0 = 0;
@@ -600,7 +622,9 @@ int run(const s12_view *views, int count, const uint16_t *const *x, int B, float
         m.esc_off = v->esc_off;
         m.esc = v->esc;
         m.x = x[i];
-        m.y = y[i];
+        m.act = act ? act[i] : 0;
+        m.y = m.act ? nullptr : static_cast<float *>(y[i]);
+        m.h = m.act ? static_cast<uint16_t *>(y[i]) : nullptr;
         m.n_esc = v->n_esc;
         m.R = static_cast<int>(R);
         m.K = static_cast<int>(K);
@@ -648,14 +672,14 @@ size_t gemv_ws_bytes(const s12_view *views, int count) {
     return pl.part_bytes + pl.cnt_bytes;
 }
 
-int launch_gemv(const s12_view *views, int count, const uint16_t *const *x, int B, float *const *y, void *ws,
-                size_t ws_bytes, uint32_t *err, cudaStream_t stream) {
+int launch_gemv(const s12_view *views, int count, const uint16_t *const *x, int B, void *const *y, const int *act,
+                void *ws, size_t ws_bytes, uint32_t *err, cudaStream_t stream) {
     int sms = 0;
     if (device_sms(&sms) != cudaSuccess) return S12_ERR_CUDA;
     const Plan pl = plan(views, count, sms);
     if (ws_bytes < pl.part_bytes + pl.cnt_bytes) return S12_ERR_CAPACITY;
-    return err ? run<true>(views, count, x, B, y, ws, err, pl, stream)
-               : run<false>(views, count, x, B, y, ws, err, pl, stream);
+    return err ? run<true>(views, count, x, B, y, act, ws, err, pl, stream)
+               : run<false>(views, count, x, B, y, act, ws, err, pl, stream);
 }
 
 }  // namespace s12

@@ -193,8 +193,12 @@ size_t s12_gemv_multi_ws_bytes(const s12_view *views, int count, int B) {
     return gemv_ws_bytes(views, count);
 }
 
-int s12_gemv_multi(const s12_view *views, int count, const uint16_t *const *x, int B, float *const *y, void *ws,
-                   size_t ws_bytes, uint32_t *err_flag, void *stream) {
+namespace {
+// Checks shared by the GEMV calls (every entry, before any launch), then the
+// launch.  act[i] == 1 marks a SwiGLU entry: interleaved gate/up rows
+// (a multiple of 16) and a BF16 output of half the rows.
+int gemv_group(const s12_view *views, int count, const uint16_t *const *x, int B, void *const *y, const int *act,
+               void *ws, size_t ws_bytes, uint32_t *err_flag, void *stream) {
     if (!views || !x || !y || !ws) return S12_ERR_ARG;
     if (count < 1 || count > S12_GEMV_MAX_PROBLEMS || B < 1 || B > S12_GEMV_MAX_BATCH) return S12_ERR_SHAPE;
     for (int i = 0; i < count; ++i) {
@@ -202,10 +206,31 @@ int s12_gemv_multi(const s12_view *views, int count, const uint16_t *const *x, i
         if (rc != S12_OK) return rc;
         if (!x[i] || !y[i]) return S12_ERR_ARG;
         if (views[i].rows > 0x7FFFFFFFull || views[i].cols > 0x7FFFFFFFull) return S12_ERR_SHAPE;
-        if (!aligned16(x[i]) || !aligned4(y[i])) return S12_ERR_ALIGN;
+        const bool swiglu = act && act[i] == 1;
+        if (act && act[i] != 0 && act[i] != 1) return S12_ERR_ARG;
+        if (swiglu && views[i].rows % 16 != 0) return S12_ERR_SHAPE;
+        if (!aligned16(x[i]) || (swiglu ? (reinterpret_cast<uintptr_t>(y[i]) & 1) != 0 : !aligned4(y[i])))
+            return S12_ERR_ALIGN;
     }
     if (!aligned16(ws) || (err_flag && !aligned4(err_flag))) return S12_ERR_ALIGN;
-    return launch_gemv(views, count, x, B, y, ws, ws_bytes, err_flag, static_cast<cudaStream_t>(stream));
+    return launch_gemv(views, count, x, B, y, act, ws, ws_bytes, err_flag, static_cast<cudaStream_t>(stream));
+}
+}  // namespace
+
+int s12_gemv_multi(const s12_view *views, int count, const uint16_t *const *x, int B, float *const *y, void *ws,
+                   size_t ws_bytes, uint32_t *err_flag, void *stream) {
+    void *out[S12_GEMV_MAX_PROBLEMS];
+    if (!y || count < 1 || count > S12_GEMV_MAX_PROBLEMS) return y ? S12_ERR_SHAPE : S12_ERR_ARG;
+    for (int i = 0; i < count; ++i) out[i] = y[i];
+    return gemv_group(views, count, x, B, out, nullptr, ws, ws_bytes, err_flag, stream);
+}
+
+int s12_gemv_swiglu(const s12_view *v, const uint16_t *x, int B, uint16_t *h, void *ws, size_t ws_bytes,
+                    uint32_t *err_flag, void *stream) {
+    if (!v || !x || !h || !ws) return S12_ERR_ARG;
+    void *out[1] = {h};
+    const int act[1] = {1};
+    return gemv_group(v, 1, &x, B, out, act, ws, ws_bytes, err_flag, stream);
 }
 
 int s12_gemv(const s12_view *v, const uint16_t *x, int B, float *y, void *ws, size_t ws_bytes, uint32_t *err_flag,

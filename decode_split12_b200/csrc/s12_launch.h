@@ -25,8 +25,10 @@ int make_tmap_bf16_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64
 
 int launch_decode(const s12_view *v, uint16_t *out, uint32_t *err, cudaStream_t stream);
 size_t gemv_ws_bytes(const s12_view *views, int count);
-int launch_gemv(const s12_view *views, int count, const uint16_t *const *x, int B, float *const *y, void *ws,
-                size_t ws_bytes, uint32_t *err, cudaStream_t stream);
+// y[i]: float* (B x rows) when act is null or act[i] == 0; uint16_t* BF16
+// (B x rows/2) when act[i] == 1 (SwiGLU of interleaved gate/up rows).
+int launch_gemv(const s12_view *views, int count, const uint16_t *const *x, int B, void *const *y, const int *act,
+                void *ws, size_t ws_bytes, uint32_t *err, cudaStream_t stream);
 int launch_bf16_gemv(const uint16_t *w, int64_t rows, int64_t cols, const uint16_t *x, int B, float *y,
                      cudaStream_t stream);
 size_t encode_ws_bytes(int64_t rows, int64_t cols);

@@ -35,7 +35,7 @@ S12_FLAG_TIMEOUT = 8
 EXPORTED = (
     "s12_error_string", "s12_device_check", "s12_container_bytes", "s12_encode_ws_bytes", "s12_encode",
     "s12_open", "s12_decode", "s12_gemv_ws_bytes", "s12_gemv", "s12_gemv_multi_ws_bytes", "s12_gemv_multi",
-    "s12_gemv_noalloc", "s12_gemm_ws_bytes", "s12_gemm_skinny", "s12_gemm_multi_ws_bytes",
+    "s12_gemv_noalloc", "s12_gemv_swiglu", "s12_gemm_ws_bytes", "s12_gemm_skinny", "s12_gemm_multi_ws_bytes",
     "s12_gemm_skinny_multi", "s12_stats_ws_bytes",
     "s12_stats", "s12_bf16_gemv",
 )
@@ -102,6 +102,8 @@ def _lib() -> C.CDLL:
         lib.s12_gemv_multi.restype = C.c_int
         lib.s12_gemv_noalloc.argtypes = [C.POINTER(View), _P, C.c_int, _P, _P, _P]
         lib.s12_gemv_noalloc.restype = C.c_int
+        lib.s12_gemv_swiglu.argtypes = [C.POINTER(View), _P, C.c_int, _P, _P, _SZ, _P, _P]
+        lib.s12_gemv_swiglu.restype = C.c_int
         lib.s12_gemv.restype = C.c_int
         lib.s12_gemm_ws_bytes.argtypes = [C.POINTER(View), C.c_int]
         lib.s12_gemm_ws_bytes.restype = _SZ
@@ -286,6 +288,32 @@ def s12_gemv_noalloc(view: View, x: torch.Tensor, y: torch.Tensor | None = None,
     _check(_lib().s12_gemv_noalloc(C.byref(view), _dptr(x), B, _dptr(y), _dptr(err_flag), _stream(stream)),
            "s12_gemv_noalloc")
     return y
+
+
+def interleave_gate_up(w_gate: torch.Tensor, w_up: torch.Tensor) -> torch.Tensor:
+    """The row order s12_gemv_swiglu expects: F x K gate and up matrices
+    (F a multiple of 8) into one 2F x K matrix whose rows 16i .. 16i+7 are
+    gate rows 8i .. 8i+7 and rows 16i+8 .. 16i+15 the up rows with the same
+    indices.  A one-time weight preparation, done before encoding."""
+    if w_gate.shape != w_up.shape or w_gate.dim() != 2 or w_gate.shape[0] % 8:
+        raise ValueError("gate and up must be F x K with F a multiple of 8")
+    F, K = w_gate.shape
+    return torch.stack([w_gate.reshape(F // 8, 8, K), w_up.reshape(F // 8, 8, K)], dim=1).reshape(2 * F, K)
+
+
+def s12_gemv_swiglu(view: View, x: torch.Tensor, h: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                    err_flag: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """h = silu(W_gate x) * (W_up x) as BF16 bits (B x rows/2), from one
+    container of interleaved gate/up rows (see interleave_gate_up)."""
+    x = _u16(x)
+    B = x.shape[0] if x.dim() == 2 else 1
+    if h is None:
+        h = torch.empty((B, view.rows // 2), dtype=torch.int16, device=x.device)
+    if ws is None:
+        ws = torch.zeros(max(s12_gemv_ws_bytes(view, B), 256), dtype=torch.uint8, device=x.device)
+    _check(_lib().s12_gemv_swiglu(C.byref(view), _dptr(x), B, _dptr(h), _dptr(ws), ws.numel(), _dptr(err_flag),
+                                  _stream(stream)), "s12_gemv_swiglu")
+    return h
 
 
 def s12_gemm_ws_bytes(view: View, M: int) -> int:

@@ -213,6 +213,27 @@ size_t s12_gemv_multi_ws_bytes(const s12_view *views, int count, int B);
 int s12_gemv_multi(const s12_view *views, int count, const uint16_t *const *x, int B, float *const *y,
                    void *ws, size_t ws_bytes, uint32_t *err_flag, void *stream);
 
+/* Fused decode-GEMV with a SwiGLU epilogue, for a gated MLP's gate and up
+ * projections (F rows each): h[b][f] = silu(g[b][f]) * u[b][f], where
+ * g = W_gate x_b, u = W_up x_b and silu(t) = t / (1 + exp(-t)), rounded to
+ * BF16 (round to nearest even).
+ *   v:  ONE container of 2F rows that interleaves the two matrices in
+ *       blocks of 8 rows: rows 16i .. 16i+7 are gate rows 8i .. 8i+7 and
+ *       rows 16i+8 .. 16i+15 are up rows 8i .. 8i+7 (so 2F must be a
+ *       multiple of 16, else S12_ERR_SHAPE).  The Python binding's
+ *       interleave_gate_up builds that matrix before encoding.
+ *   x:  device BF16, B x cols; 1 <= B <= 8.
+ *   h:  device BF16, B x F row-major (2-byte alignment), overwritten.  It is
+ *       the input of the down projection, so the gate and up outputs never
+ *       go to memory.
+ *   ws: as for s12_gemv (size s12_gemv_ws_bytes(v, B)).
+ * The warp-level product gives each lane rows r and r + 8 of a 16-row group,
+ * which here are gate row f and up row f: the activation is applied where
+ * the sums are stored ([W] "What does 'lossless' mean for LLM weights?":
+ * decode and use the weights at once; the epilogue is this build's own). */
+int s12_gemv_swiglu(const s12_view *v, const uint16_t *x, int B, uint16_t *h, void *ws, size_t ws_bytes,
+                    uint32_t *err_flag, void *stream);
+
 /* s12_gemv for callers that cannot allocate device memory (no counterpart
  * in the pages: it exists for integration, not for the method).  Examples are
  * a plugin whose host engine owns all device memory through its own

@@ -58,6 +58,8 @@ def _bind(lib: C.CDLL) -> C.CDLL:
     lib.oracle_gemv_f64.restype = C.c_int
     lib.oracle_gemv_rows_f64.argtypes = [_P, _U64, _P, _I64, _P, _I64, _P, _P]
     lib.oracle_gemv_rows_f64.restype = C.c_int
+    lib.oracle_silu_mul_f64.argtypes = [_P, _P, _I64, _P]
+    lib.oracle_silu_mul_f64.restype = C.c_int
     lib.oracle_stats.argtypes = [_P, _U64, _P]
     lib.oracle_stats.restype = C.c_int
     lib.oracle_bf16_to_double.argtypes = [C.c_uint16]
@@ -185,6 +187,23 @@ class Oracle:
         _check(self.lib.oracle_gemv_rows_f64(_ptr(blob), blob.size, _ptr(x), m, _ptr(idx), idx.size,
                                              _ptr(y), _ptr(s)), "gemv_rows")
         return y, s
+
+    def silu_mul_f64(self, g: np.ndarray, u: np.ndarray) -> np.ndarray:
+        """h = silu(g) * u elementwise (the C oracle's gated-MLP activation)."""
+        g = np.ascontiguousarray(g, dtype=np.float64)
+        u = np.ascontiguousarray(u, dtype=np.float64)
+        assert g.shape == u.shape
+        h = np.zeros_like(g)
+        _check(self.lib.oracle_silu_mul_f64(_ptr(g), _ptr(u), g.size, _ptr(h)), "silu_mul")
+        return h
+
+    def swiglu_f64(self, blob_gate: np.ndarray, blob_up: np.ndarray, x: np.ndarray):
+        """Gated MLP input side: g = W_gate x, u = W_up x (FP64 GEMVs of two
+        separate containers), h = silu(g) * u.  Returns h, g, u and the
+        tolerance scales s_g, s_u (all m x F)."""
+        g, s_g = self.gemv_f64(blob_gate, x)
+        u, s_u = self.gemv_f64(blob_up, x)
+        return self.silu_mul_f64(g, u), g, u, s_g, s_u
 
     def stats(self, blob: np.ndarray) -> dict:
         blob = np.ascontiguousarray(blob, dtype=np.uint8)

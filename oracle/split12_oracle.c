@@ -394,6 +394,17 @@ int oracle_gemv_rows_f64(const uint8_t *blob, uint64_t bytes, const uint16_t *x,
     return rc;
 }
 
+/* Gated-MLP activation for the SwiGLU epilogue of the fused GEMV: with
+ * g = W_gate x and u = W_up x computed as above (in FP64),
+ *     h = silu(g) * u,   silu(t) = t / (1 + exp(-t)),
+ * elementwise over n values.  The pages name fused epilogues for decode
+ * kernels but not an activation; this is the standard gated-MLP form. */
+int oracle_silu_mul_f64(const double *g, const double *u, int64_t n, double *h) {
+    if (!g || !u || !h || n < 0) return ORACLE_ERR_ARG;
+    for (int64_t i = 0; i < n; i++) h[i] = g[i] / (1.0 + exp(-g[i])) * u[i];
+    return ORACLE_OK;
+}
+
 /* ---------------------------------------------------------------------- */
 /* Statistics ([M] section 1: exponent and mantissa entropy of BF16 weights;
  * [T] key points: 12-bit rate, escape rate).                               */

@@ -253,6 +253,44 @@ def test_gemv_matches_independent_fp64(oracle):
 
 # ---------------------------------------------------------------- corruption
 
+def test_silu_mul_textbook_values(oracle):
+    """The gated-MLP activation h = silu(g) * u against values fixed by the
+    logistic function itself: silu(0) = 0; silu(1) = e / (1 + e); silu(t)
+    -> t for large t and -> 0 for large negative t; silu(t) - silu(-t) = t
+    (because the logistic satisfies s(t) + s(-t) = 1).  A flipped sign in
+    the exponent, a dropped factor or swapped operands fails one of them."""
+    e = math.e
+    g = np.array([0.0, 1.0, 1.0, 2.0, 64.0, -64.0, 3.5, -3.5, 0.25, -0.25])
+    u = np.array([5.0, 1.0, 2.0, 1.0, 3.0, 3.0, 1.0, 1.0, 1.0, 1.0])
+    h = oracle.silu_mul_f64(g, u)
+    assert h[0] == 0.0
+    assert h[1] == pytest.approx(e / (1 + e), rel=1e-15)
+    assert h[2] == pytest.approx(2 * e / (1 + e), rel=1e-15)          # gate 1, up 2
+    assert h[3] == pytest.approx(2 * e * e / (1 + e * e), rel=1e-15)  # gate 2, up 1: not the same
+    assert h[4] == pytest.approx(192.0, rel=1e-25)
+    assert abs(h[5]) < 1e-24
+    assert h[6] - h[7] == pytest.approx(3.5, rel=1e-15)
+    assert h[8] - h[9] == pytest.approx(0.25, rel=1e-15)
+
+
+def test_swiglu_one_hot_uses_gate_and_up_columns(oracle):
+    """x = e_j: g and u are column j of each matrix exactly, and h applies
+    the activation to the gate column only."""
+    wg = wl.normal_with_outliers(40, 256, 0.5, 0.0, 5)
+    wu = wl.normal_with_outliers(40, 256, 0.5, 0.0, 6)
+    bg, bu = oracle.encode(wg), oracle.encode(wu)
+    j = 77
+    x = np.zeros((1, 256), np.uint16)
+    x[0, j] = 0x3F80
+    h, g, u, s_g, s_u = oracle.swiglu_f64(bg, bu, x)
+    cg = wl.bf16_bits_to_f32(wg[:, j]).astype(np.float64)
+    cu = wl.bf16_bits_to_f32(wu[:, j]).astype(np.float64)
+    assert np.array_equal(g[0], cg) and np.array_equal(u[0], cu)
+    assert np.array_equal(s_g[0], np.abs(cg)) and np.array_equal(s_u[0], np.abs(cu))
+    assert np.array_equal(h[0], oracle.silu_mul_f64(cg, cu))
+    assert not np.allclose(h[0], oracle.silu_mul_f64(cu, cg))
+
+
 def test_corruption_detected(oracle):
     """Flipping bytes must make the decoder fail closed (wavect, 14-day pilot,
     step 2: inject corruption and confirm it is detected)."""
