@@ -101,3 +101,54 @@ def test_argument_checks_need_no_device(lib):
     assert lib.s12_open(bad, 1024, C.byref(v)) == s12.S12_ERR_ALIGN
     assert lib.s12_open(fake, 100, C.byref(v)) == s12.S12_ERR_CORRUPT
     assert lib.s12_bf16_gemv(fake, 4, 12, fake, 1, fake, None) == s12.S12_ERR_SHAPE
+
+
+def test_swiglu_and_gemm_group_argument_checks(lib):
+    """The SwiGLU and grouped-GEMM entry points reject bad arguments on the
+    host, before any device work: rows not a multiple of 16 for SwiGLU, an
+    odd output address, more than 16 matrices, a token count above 256."""
+    from decode_split12_b200 import s12
+    fake = C.c_void_p(0x100000)
+    v = s12.View()
+    v.rows, v.cols, v.n_tiles = 24, 128, 24
+    for f in ("container", "raw", "code", "base", "esc_off", "esc"):
+        setattr(v, f, 0x100000)
+    assert lib.s12_gemv_swiglu(C.byref(v), fake, 1, fake, fake, 1 << 20, None, None) == s12.S12_ERR_SHAPE
+    v.rows, v.n_tiles = 32, 32
+    odd = C.c_void_p(0x100001)
+    assert lib.s12_gemv_swiglu(C.byref(v), fake, 1, odd, fake, 1 << 20, None, None) == s12.S12_ERR_ALIGN
+    assert lib.s12_gemv_swiglu(C.byref(v), fake, 9, fake, fake, 1 << 20, None, None) == s12.S12_ERR_SHAPE
+    assert lib.s12_gemv_swiglu(C.byref(v), fake, 1, None, fake, 1 << 20, None, None) == s12.S12_ERR_ARG
+    views = (s12.View * 17)(*([v] * 17))
+    xs = (C.c_void_p * 17)(*([0x100000] * 17))
+    ys = (C.c_void_p * 17)(*([0x100000] * 17))
+    ms = (C.c_int * 17)(*([16] * 17))
+    assert lib.s12_gemm_skinny_multi(views, 17, xs, ms, ys, fake, 1 << 20, None, None) == s12.S12_ERR_ARG
+    ms[1] = 257
+    assert lib.s12_gemm_skinny_multi(views, 2, xs, ms, ys, fake, 1 << 20, None, None) == s12.S12_ERR_SHAPE
+    assert lib.s12_gemm_multi_ws_bytes(views, 2, ms) == 0
+    ms[1] = 0
+    assert lib.s12_gemm_skinny_multi(views, 2, xs, ms, ys, fake, 1 << 20, None, None) == s12.S12_ERR_SHAPE
+
+
+def test_interleave_gate_up_row_order():
+    """Rows 16i .. 16i+7 of the interleaved matrix are gate rows 8i .. 8i+7
+    and rows 16i+8 .. 16i+15 the up rows with the same indices, which is the
+    pairing the SwiGLU epilogue's lanes rely on (a lane holds rows r and
+    r + 8 of each 16-row group)."""
+    import torch
+
+    from decode_split12_b200 import s12
+    F, K = 24, 256
+    gate = torch.arange(F * K, dtype=torch.int32).reshape(F, K).to(torch.int16)
+    up = (torch.arange(F * K, dtype=torch.int32).reshape(F, K) + 30000).to(torch.int16)
+    wi = s12.interleave_gate_up(gate, up)
+    assert wi.shape == (2 * F, K)
+    for r in range(2 * F):
+        grp, within = divmod(r, 16)
+        src = gate if within < 8 else up
+        assert torch.equal(wi[r], src[8 * grp + within % 8]), r
+    with pytest.raises(ValueError):
+        s12.interleave_gate_up(gate[:20], up[:20])
+    with pytest.raises(ValueError):
+        s12.interleave_gate_up(gate, up[:16])
