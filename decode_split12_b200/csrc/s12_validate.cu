@@ -1,0 +1,132 @@
+// s12_validate.cu -- host-side container validation and per-plane hashes.
+//
+// "Lossless LLM Weight Compression vs 8-bit GGUF", section "A 14-day
+// production-readiness pilot": inject corruption and confirm that it is
+// detected rather than decoded into wrong weights.  The kernels already raise
+// err_flag bits when they meet inconsistent escape data; these calls check a
+// whole container in host memory before it is trusted (for instance after it
+// is read from disk), and give 64-bit hashes of its planes so that bytes
+// without redundancy (raw bytes, escape values) can be checked against hashes
+// stored at encode time.
+//
+// A container is valid when the header is well formed, the bytes cover every
+// plane, esc_off starts at 0 and ends at n_esc, and every tile has
+// non-decreasing offsets within the stream, a base of at most 241 and exactly
+// as many code-15 nibbles as its offsets span.  Non-zero padding does not
+// make a container invalid (nothing reads it); it is reported as a note.
+#include <cstring>
+
+#include "s12_device.cuh"
+#include "s12_launch.h"
+
+namespace s12 {
+namespace {
+
+uint32_t rd32(const uint8_t *p) {
+    return uint32_t(p[0]) | uint32_t(p[1]) << 8 | uint32_t(p[2]) << 16 | uint32_t(p[3]) << 24;
+}
+uint64_t rd64(const uint8_t *p) { return uint64_t(rd32(p)) | uint64_t(rd32(p + 4)) << 32; }
+
+// FNV-1a, 64-bit: offset basis 0xcbf29ce484222325, prime 0x100000001b3.
+uint64_t fnv1a64(const uint8_t *p, uint64_t n) {
+    uint64_t h = 0xcbf29ce484222325ull;
+    for (uint64_t i = 0; i < n; ++i) {
+        h ^= p[i];
+        h *= 0x100000001b3ull;
+    }
+    return h;
+}
+
+bool any_nonzero(const uint8_t *p, uint64_t n) {
+    for (uint64_t i = 0; i < n; ++i)
+        if (p[i]) return true;
+    return false;
+}
+
+// Header checks shared by both calls; fills the geometry.
+int parse_header(const uint8_t *c, size_t bytes, Geometry *g) {
+    if (bytes < kHeaderBytes) return S12_BAD_SIZE;
+    if (std::memcmp(c, "S12\0", 4) != 0 || rd32(c + 4) != 1 || rd32(c + 24) != static_cast<uint32_t>(kTile) ||
+        rd32(c + 28) != 0)
+        return S12_BAD_HEADER;
+    for (int i = 40; i < 64; ++i)
+        if (c[i]) return S12_BAD_HEADER;
+    const uint64_t rows = rd64(c + 8), cols = rd64(c + 16), n_esc = rd64(c + 32);
+    if (rows == 0 || cols == 0 || cols % kTile) return S12_BAD_HEADER;
+    if (rows >= (uint64_t(1) << 32) || cols >= (uint64_t(1) << 32) || rows * cols >= (uint64_t(1) << 32))
+        return S12_BAD_HEADER;
+    if (n_esc > rows * cols) return S12_BAD_HEADER;
+    *g = geometry(rows, cols, n_esc);
+    if (g->total > bytes) return S12_BAD_SIZE;
+    return 0;
+}
+
+}  // namespace
+}  // namespace s12
+
+using namespace s12;
+
+extern "C" uint64_t s12_fnv1a64(const void *data, size_t bytes) {
+    return data ? fnv1a64(static_cast<const uint8_t *>(data), bytes) : fnv1a64(nullptr, 0);
+}
+
+extern "C" int s12_validate_host(const void *container, size_t bytes, s12_report *out) {
+    if (!container || !out) return S12_ERR_ARG;
+    std::memset(out, 0, sizeof *out);
+    const uint8_t *c = static_cast<const uint8_t *>(container);
+    Geometry g;
+    const int bad = parse_header(c, bytes, &g);
+    if (bad) {
+        out->problem = static_cast<uint32_t>(bad);
+        return S12_ERR_CORRUPT;
+    }
+    const uint8_t *code = c + g.off_code, *base = c + g.off_base, *off = c + g.off_esc_off;
+    if (rd32(off) != 0 || rd32(off + 4 * g.n_tiles) != g.n_esc) {
+        out->problem = S12_BAD_OFFSETS;
+        return S12_ERR_CORRUPT;
+    }
+    for (uint64_t t = 0; t < g.n_tiles; ++t) {
+        const uint32_t lo = rd32(off + 4 * t), hi = rd32(off + 4 * (t + 1));
+        uint32_t n15 = 0;
+        for (int k = 0; k < kTile / 2; ++k) {
+            const uint8_t b = code[t * (kTile / 2) + k];
+            n15 += ((b & 0x0F) == 0x0F) + ((b >> 4) == 0x0F);
+        }
+        out->n_esc_counted += n15;
+        uint32_t problem = 0;
+        if (hi < lo || hi > g.n_esc)
+            problem = S12_BAD_TILE_OFFSETS;
+        else if (base[t] > kMaxBase)
+            problem = S12_BAD_BASE;
+        else if (n15 != hi - lo)
+            problem = S12_BAD_ESC_COUNT;
+        if (problem) {
+            out->problem = problem;
+            out->tile = t;
+            return S12_ERR_CORRUPT;
+        }
+    }
+    // padding after the 64 header bytes in use and after every plane
+    const uint64_t ends[6][2] = {{64, g.off_raw},
+                                 {g.off_raw + g.rows * g.cols, g.off_code},
+                                 {g.off_code + g.rows * g.cols / 2, g.off_base},
+                                 {g.off_base + g.n_tiles, g.off_esc_off},
+                                 {g.off_esc_off + 4 * (g.n_tiles + 1), g.off_esc},
+                                 {g.off_esc + 2 * g.n_esc, g.total}};
+    for (const auto &e : ends)
+        if (any_nonzero(c + e[0], e[1] - e[0])) out->notes |= S12_NOTE_PADDING;
+    return S12_OK;
+}
+
+extern "C" int s12_plane_hashes_host(const void *container, size_t bytes, uint64_t out[5]) {
+    if (!container || !out) return S12_ERR_ARG;
+    const uint8_t *c = static_cast<const uint8_t *>(container);
+    Geometry g;
+    if (parse_header(c, bytes, &g)) return S12_ERR_CORRUPT;
+    out[0] = fnv1a64(c + g.off_raw, g.rows * g.cols);
+    out[1] = fnv1a64(c + g.off_code, g.rows * g.cols / 2);
+    out[2] = fnv1a64(c + g.off_base, g.n_tiles);
+    out[3] = fnv1a64(c + g.off_esc_off, 4 * (g.n_tiles + 1));
+    out[4] = fnv1a64(c + g.off_esc, 2 * g.n_esc);
+    return S12_OK;
+}

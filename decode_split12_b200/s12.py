@@ -12,6 +12,7 @@ from __future__ import annotations
 
 import ctypes as C
 import os
+import numpy as np
 
 import torch
 
@@ -36,7 +37,7 @@ EXPORTED = (
     "s12_error_string", "s12_device_check", "s12_container_bytes", "s12_encode_ws_bytes", "s12_encode",
     "s12_open", "s12_decode", "s12_gemv_ws_bytes", "s12_gemv", "s12_gemv_multi_ws_bytes", "s12_gemv_multi",
     "s12_gemv_noalloc", "s12_gemv_swiglu", "s12_gemm_ws_bytes", "s12_gemm_skinny", "s12_gemm_multi_ws_bytes",
-    "s12_gemm_skinny_multi", "s12_stats_ws_bytes",
+    "s12_gemm_skinny_multi", "s12_validate_host", "s12_plane_hashes_host", "s12_fnv1a64", "s12_stats_ws_bytes",
     "s12_stats", "s12_bf16_gemv",
 )
 
@@ -109,6 +110,12 @@ def _lib() -> C.CDLL:
         lib.s12_gemm_ws_bytes.restype = _SZ
         lib.s12_gemm_skinny.argtypes = [C.POINTER(View), _P, C.c_int, _P, _P, _SZ, _P, _P]
         lib.s12_gemm_skinny.restype = C.c_int
+        lib.s12_validate_host.argtypes = [_P, _SZ, C.POINTER(Report)]
+        lib.s12_validate_host.restype = C.c_int
+        lib.s12_plane_hashes_host.argtypes = [_P, _SZ, C.POINTER(C.c_uint64)]
+        lib.s12_plane_hashes_host.restype = C.c_int
+        lib.s12_fnv1a64.argtypes = [_P, _SZ]
+        lib.s12_fnv1a64.restype = C.c_uint64
         lib.s12_gemm_multi_ws_bytes.argtypes = [C.POINTER(View), C.c_int, C.POINTER(C.c_int)]
         lib.s12_gemm_multi_ws_bytes.restype = _SZ
         lib.s12_gemm_skinny_multi.argtypes = [C.POINTER(View), C.c_int, C.POINTER(_P), C.POINTER(C.c_int),
@@ -380,3 +387,38 @@ def s12_gemm_skinny_multi(views, xs, ys=None, ws: torch.Tensor | None = None, er
     _check(_lib().s12_gemm_skinny_multi(arr, len(views), xp, ma, yp, _dptr(ws), ws.numel(), _dptr(err_flag),
                                         _stream(stream)), "s12_gemm_skinny_multi")
     return ys
+
+
+class Report(C.Structure):
+    _fields_ = [("problem", C.c_uint32), ("notes", C.c_uint32), ("tile", C.c_uint64), ("n_esc_counted", C.c_uint64)]
+
+
+S12_BAD_NAMES = {1: "header", 2: "size", 3: "offsets", 4: "tile_offsets", 5: "base", 6: "esc_count"}
+
+
+def _host_bytes(container) -> np.ndarray:
+    a = container.cpu().numpy() if isinstance(container, torch.Tensor) else np.asarray(container)
+    return np.ascontiguousarray(a).view(np.uint8).reshape(-1)
+
+
+def s12_validate_host(container):
+    """Validate a container (host array or tensor, copied to host if needed).
+    Returns (status, report) with report a dict of the first problem found."""
+    b = _host_bytes(container)
+    rep = Report()
+    rc = _lib().s12_validate_host(b.ctypes.data_as(C.c_void_p), b.size, C.byref(rep))
+    return rc, {"problem": S12_BAD_NAMES.get(rep.problem), "notes": int(rep.notes), "tile": int(rep.tile),
+                "n_esc_counted": int(rep.n_esc_counted)}
+
+
+def s12_plane_hashes_host(container):
+    """FNV-1a 64-bit hashes of the raw, code, base, esc_off and esc planes."""
+    b = _host_bytes(container)
+    out = (C.c_uint64 * 5)()
+    _check(_lib().s12_plane_hashes_host(b.ctypes.data_as(C.c_void_p), b.size, out), "s12_plane_hashes_host")
+    return [int(v) for v in out]
+
+
+def s12_fnv1a64(data: bytes) -> int:
+    buf = C.create_string_buffer(bytes(data), len(data))
+    return int(_lib().s12_fnv1a64(C.cast(buf, C.c_void_p), len(data)))

@@ -307,6 +307,43 @@ size_t s12_stats_ws_bytes(void);
  * decoded weights.  Runs a histogram kernel and SYNCHRONISES `stream`. */
 int s12_stats(const s12_view *v, s12_stats_t *out, void *ws, size_t ws_bytes, void *stream);
 
+/* ---- host-side validation and plane hashes ([W] "A 14-day
+ * production-readiness pilot": inject corruption and confirm that it is
+ * detected, not decoded into wrong weights) ---- */
+
+#define S12_BAD_HEADER 1u       /* magic, version, tile, flags, reserved bytes or shape */
+#define S12_BAD_SIZE 2u         /* fewer bytes than the header's planes need          */
+#define S12_BAD_OFFSETS 3u      /* esc_off[0] != 0 or esc_off[n_tiles] != n_esc       */
+#define S12_BAD_TILE_OFFSETS 4u /* a tile's offsets decrease or pass n_esc            */
+#define S12_BAD_BASE 5u         /* a tile base above 241                              */
+#define S12_BAD_ESC_COUNT 6u    /* a tile's code-15 count != its offset span          */
+#define S12_NOTE_PADDING 1u     /* a padding byte is not zero (nothing reads it)      */
+
+typedef struct s12_report {
+    uint32_t problem;       /* S12_BAD_* of the first problem found, 0 if valid */
+    uint32_t notes;         /* S12_NOTE_* bits (do not make the container invalid) */
+    uint64_t tile;          /* the tile of a per-tile problem                   */
+    uint64_t n_esc_counted; /* code-15 nibbles in the tiles checked             */
+} s12_report;
+
+/* Check a whole container in HOST memory (for instance a file read before
+ * it is copied to the device): S12_OK when it is valid, S12_ERR_CORRUPT with
+ * *out describing the first problem otherwise (S12_ERR_ARG for NULLs).  A
+ * valid container decodes without any err_flag bit.  Raw bytes and escape
+ * values carry no redundancy, so a change there is only caught by
+ * s12_plane_hashes_host. */
+int s12_validate_host(const void *container, size_t bytes, s12_report *out);
+
+/* 64-bit FNV-1a hashes of the exact bytes of the five planes, in the order
+ * raw, code, base, esc_off, esc (padding excluded), of a container in HOST
+ * memory with a valid header.  Any change of a single byte changes its
+ * plane's hash.  Store them at encode time and compare after loading. */
+int s12_plane_hashes_host(const void *container, size_t bytes, uint64_t out[5]);
+
+/* FNV-1a 64-bit hash of `bytes` bytes (offset basis 0xcbf29ce484222325,
+ * prime 0x100000001b3), the function s12_plane_hashes_host uses. */
+uint64_t s12_fnv1a64(const void *data, size_t bytes);
+
 /* ---- uncompressed baseline ---- */
 
 /* Plain BF16 GEMV, the comparison point for s12_gemv: y[b][n] =

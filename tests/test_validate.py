@@ -1,0 +1,139 @@
+"""Host-side container validation and plane hashes, with a corruption-
+injection suite (no GPU needed): every corruption is judged the same way by
+the library's validator and by the oracle's decoder (an independent
+implementation of the container definition), with the expected problem
+named; byte changes that leave the structure intact (raw bytes, escape
+values) are caught by the plane hashes instead."""
+import numpy as np
+import pytest
+
+from decode_split12_b200 import s12
+from decode_split12_b200 import workloads as wl
+
+ALIGN = 256
+
+
+def _pad(n):
+    return (n + ALIGN - 1) // ALIGN * ALIGN
+
+
+def _planes(rows, cols, n_esc):
+    """Byte ranges of the planes, from the container layout (256-byte header,
+    then raw, code, base, esc_off, esc, each padded to 256 bytes)."""
+    n_t = rows * cols // 128
+    sizes = [rows * cols, rows * cols // 2, n_t, 4 * (n_t + 1), 2 * n_esc]
+    out, off = [], ALIGN
+    for sz in sizes:
+        out.append((off, off + sz))
+        off += _pad(sz)
+    return out
+
+
+def test_fnv1a64_published_vectors():
+    """The FNV-1a 64-bit test vectors of the function's published
+    definition."""
+    assert s12.s12_fnv1a64(b"") == 0xCBF29CE484222325
+    assert s12.s12_fnv1a64(b"a") == 0xAF63DC4C8601EC8C
+    assert s12.s12_fnv1a64(b"foobar") == 0x85944171F73967E8
+
+
+@pytest.fixture(scope="module")
+def blob(oracle):
+    w, n = wl.escape_stress(0.02, 3, 64, 512)   # escapes in most tiles
+    b = oracle.encode(w)
+    return b, w.shape, n
+
+
+def test_valid_containers(oracle):
+    for i, (r, c) in enumerate([(1, 128), (37, 640), (64, 4096)]):
+        b = oracle.encode(wl.normal_with_outliers(r, c, 0.02, 0.01, i))
+        rc, rep = s12.s12_validate_host(b)
+        assert rc == s12.S12_OK and rep["problem"] is None and rep["notes"] == 0
+        assert rep["n_esc_counted"] == int(np.frombuffer(b[32:40].tobytes(), np.uint64)[0])
+
+
+def _corrupt_and_judge(oracle, b, mutate):
+    c = b.copy()
+    mutate(c)
+    rc, rep = s12.s12_validate_host(c)
+    orc_bad = oracle.decode_rc(c) != 0
+    assert (rc != s12.S12_OK) == orc_bad, (rc, rep)
+    return rc, rep
+
+
+def _u32_at(c, off, v):
+    c[off:off + 4] = np.frombuffer(np.uint32(v).tobytes(), np.uint8)
+
+
+def test_header_corruptions(oracle, blob):
+    b, _, _ = blob
+    cases = {
+        "magic": lambda c: c.__setitem__(1, ord("X")),
+        "version": lambda c: _u32_at(c, 4, 2),
+        "tile": lambda c: _u32_at(c, 24, 64),
+        "flags": lambda c: _u32_at(c, 28, 1),
+        "reserved": lambda c: c.__setitem__(50, 7),
+        "cols": lambda c: c.__setitem__(16, 100),
+    }
+    for name, f in cases.items():
+        rc, rep = _corrupt_and_judge(oracle, b, f)
+        assert rc == s12.S12_ERR_CORRUPT and rep["problem"] == "header", name
+
+
+def test_size_and_offset_corruptions(oracle, blob):
+    b, (rows, cols), n_esc = blob
+    (_, _), (_, _), (_, _), (o0, o1), _ = _planes(rows, cols, n_esc)
+    n_t = rows * cols // 128
+    rc, rep = _corrupt_and_judge(oracle, b[:-1], lambda c: None)
+    assert rep["problem"] == "size"
+    rc, rep = _corrupt_and_judge(oracle, b, lambda c: _u32_at(c, o0, 1))
+    assert rep["problem"] == "offsets"
+    rc, rep = _corrupt_and_judge(oracle, b, lambda c: _u32_at(c, o0 + 4 * n_t, n_esc + 1))
+    assert rep["problem"] == "offsets"
+    # a middle offset moved below its predecessor: tile t-1 now ends before it starts
+    t = n_t // 2
+    rc, rep = _corrupt_and_judge(oracle, b, lambda c: _u32_at(c, o0 + 4 * t, 0))
+    assert rc == s12.S12_ERR_CORRUPT and rep["problem"] in ("tile_offsets", "esc_count")
+    # a middle offset moved past the end of the stream
+    rc, rep = _corrupt_and_judge(oracle, b, lambda c: _u32_at(c, o0 + 4 * t, n_esc + 5))
+    assert rep["problem"] == "tile_offsets"
+
+
+def test_base_and_code_corruptions(oracle, blob):
+    b, (rows, cols), n_esc = blob
+    _, (c0, _), (b0, _), _, _ = _planes(rows, cols, n_esc)
+    rc, rep = _corrupt_and_judge(oracle, b, lambda c: c.__setitem__(b0 + 5, 242))
+    assert rep["problem"] == "base" and rep["tile"] == 5
+    # a code nibble turned into an escape, and an escape turned into a code
+    codes = b[c0:c0 + rows * cols // 2]
+    lo_nib = codes & 0x0F
+    k_plain = int(np.flatnonzero(lo_nib != 0x0F)[10])
+    k_esc = int(np.flatnonzero(lo_nib == 0x0F)[0])
+    rc, rep = _corrupt_and_judge(oracle, b, lambda c: c.__setitem__(c0 + k_plain, (c[c0 + k_plain] & 0xF0) | 0x0F))
+    assert rep["problem"] == "esc_count" and rep["tile"] == (2 * k_plain) // 128
+    rc, rep = _corrupt_and_judge(oracle, b, lambda c: c.__setitem__(c0 + k_esc, (c[c0 + k_esc] & 0xF0) | 0x03))
+    assert rep["problem"] == "esc_count" and rep["tile"] == (2 * k_esc) // 128
+
+
+def test_structure_free_bytes_caught_by_hashes(oracle, blob):
+    """A raw byte, an escape value or a padding byte changed: the container
+    stays valid for both implementations, but the changed plane's hash (and
+    only that one) differs; padding only raises the note."""
+    b, (rows, cols), n_esc = blob
+    planes = _planes(rows, cols, n_esc)
+    h0 = s12.s12_plane_hashes_host(b)
+    for i, (lo, hi) in enumerate(planes):
+        assert h0[i] == s12.s12_fnv1a64(b[lo:hi].tobytes())
+    for plane, pos in ((0, 1000), (4, 6)):
+        rc, rep = _corrupt_and_judge(oracle, b, lambda c: c.__setitem__(planes[plane][0] + pos,
+                                                                         c[planes[plane][0] + pos] ^ 0x40))
+        assert rc == s12.S12_OK
+        c = b.copy()
+        c[planes[plane][0] + pos] ^= 0x40
+        h1 = s12.s12_plane_hashes_host(c)
+        assert [h1[i] != h0[i] for i in range(5)] == [i == plane for i in range(5)]
+    assert planes[3][1] + 3 < planes[4][0]   # inside esc_off's padding
+    rc, rep = _corrupt_and_judge(oracle, b, lambda c: c.__setitem__(planes[3][1] + 3, 9))
+    assert rc == s12.S12_OK and rep["notes"] == 1
+    rc, rep = _corrupt_and_judge(oracle, b, lambda c: c.__setitem__(100, 1))   # header padding
+    assert rc == s12.S12_OK and rep["notes"] == 1
