@@ -109,42 +109,12 @@ __device__ __forceinline__ void bar_expect_tx(uint32_t bar, uint32_t bytes) {
 }
 
 // Bounded wait for phase `parity`; false after about a second.
-#ifndef S12_GEMM_WAIT_MODE
-#define S12_GEMM_WAIT_MODE 0
-#endif
-
-__device__ __forceinline__ bool bar_test(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
 __device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity) {
-#if S12_GEMM_WAIT_MODE == 1
-    if (bar_test(bar, parity)) return true;
-    const long long t0 = clock64();
-    while (!bar_test(bar, parity))
-        if (clock64() - t0 > kWaitCycles) return false;
-    return true;
-#elif S12_GEMM_WAIT_MODE == 2
-    if (mbar_try_wait_hint(bar, parity, 20u)) return true;
-    const long long t0 = clock64();
-    while (!mbar_try_wait_hint(bar, parity, 20u))
-        if (clock64() - t0 > kWaitCycles) return false;
-    return true;
-#else
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity))
         if (clock64() - t0 > kWaitCycles) return false;
     return true;
-#endif
 }
 
 __device__ __forceinline__ void tma2d(uint32_t dst, const CUtensorMap *tm, int c0, int c1, uint32_t bar,

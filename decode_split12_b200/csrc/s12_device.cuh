@@ -88,34 +88,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// try_wait that lets the hardware suspend the thread for up to `ns`
-// nanoseconds while the phase is pending (no issue slots burnt spinning).
-__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity, uint32_t ns) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity), "r"(ns)
-        : "memory");
-    return ok != 0;
-}
-
 // Wait for the phase with the given parity to complete.  Returns false (and
 // raises S12_FLAG_TIMEOUT) if it does not within kWaitCycles.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t *err) {
     const uint32_t a = smem_addr(bar);
     if (mbar_try_wait(a, parity)) return true;
     const long long t0 = clock64();
-#ifndef S12_WAIT_MODE
-#define S12_WAIT_MODE 1
-#endif
-#if S12_WAIT_MODE == 0
-    while (!mbar_try_wait_hint(a, parity, 20000u)) {
-#else
     while (!mbar_try_wait(a, parity)) {
-#endif
         if (clock64() - t0 > kWaitCycles) {
             raise_flag(err, S12_FLAG_TIMEOUT);
             return false;
