@@ -28,8 +28,10 @@
 // refills it as soon as the lanes have read it into registers.  The ring
 // keeps several blocks in flight per warp at no register cost, so 16 warps
 // fit on an SM.  The per-tile base and escape offsets are read with plain
-// loads two blocks ahead, and the first escape value of a tile that has
-// escapes is fetched one block ahead, so escapes rarely stall a warp.
+// loads two blocks ahead.  Escape values are read when a block needs them:
+// prefetching each tile's first escape one block ahead cost more in
+// per-block work and registers than the load it hid (the layer ran 7.5 %
+// slower with it).
 //
 // Work split (stream-K).  Blocks are numbered row-group-major (16-row group,
 // then tile column) and dealt to all warps of the grid in equal contiguous
@@ -205,14 +207,6 @@ __device__ __forceinline__ Meta load_meta_next(const Problem &m_, Pos ps, int g,
     return m;
 }
 
-// The first escape value of a tile with escapes (0 otherwise), fetched ahead
-// of its use.
-__device__ __forceinline__ uint32_t first_escape(const Problem &m_, uint32_t lo, uint32_t hi) {
-    uint32_t v = 0;
-    if (lo < hi && lo < m_.n_esc) v = __ldg(m_.esc + lo);
-    return v;
-}
-
 // First block of warp unit u's range.
 __device__ __forceinline__ long long unit_start(long long u, long long n_blocks, int n_units) {
     return u * n_blocks / n_units;
@@ -348,8 +342,8 @@ __device__ __forceinline__ EscRow prepare_row(uint4 c, uint32_t lo, uint32_t hi,
 // carry into the next byte, so such chunks are decoded again with the
 // escape nibbles cleared first.
 __device__ __forceinline__ void fix_chunk(uint32_t (&w)[8], uint4 raw, uint2 code, uint32_t base, uint32_t idx,
-                                          uint32_t limit, uint32_t first, uint32_t first_val,
-                                          const uint16_t *__restrict__ esc, uint32_t *err, uint32_t sc) {
+                                          uint32_t limit, const uint16_t *__restrict__ esc, uint32_t *err,
+                                          uint32_t sc) {
     const uint2 m = esc_mask(code);
     if (base > static_cast<uint32_t>(kMaxBase - 1))
         decode16(raw, make_uint2(clear_escapes(code.x, m.x), clear_escapes(code.y, m.y)), base * 0x01010101u, w);
@@ -365,7 +359,7 @@ __device__ __forceinline__ void fix_chunk(uint32_t (&w)[8], uint4 raw, uint2 cod
         mm &= mm - 1;
         uint32_t v = 0;
         if (idx < limit)
-            v = idx == first ? first_val : __ldg(esc + idx);
+            v = __ldg(esc + idx);
         else
             raise_flag(err, S12_FLAG_ESC_RANGE);
         ++idx;
@@ -459,7 +453,6 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_tma_kernel(const __grid_c
     Meta m0 = load_meta(pr.prob[pm.p], pm, g), m1 = m0;
     advance(pm, pr);
     if (nb > 1) m1 = load_meta(pr.prob[pm.p], pm, g);
-    uint32_t fvA = first_escape(pr.prob[p0.p], m0.loA, m0.hiA), fvB = first_escape(pr.prob[p0.p], m0.loB, m0.hiB);
     float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};  // one chain per half
     Pos cur = p0;
     const long long G0 = group_id(pr, p0);
@@ -467,19 +460,11 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_tma_kernel(const __grid_c
     uint32_t parity = 0;
     bool ok = true;
     for (int i = 0; i < nb; ++i) {
-        // metadata two blocks ahead, the next block's first escapes one ahead
+        // metadata two blocks ahead
         Meta m2 = m1;
         if (i + 2 < nb) {
             advance(pm, pr);
             m2 = pm.j > 0 ? load_meta_next(pr.prob[pm.p], pm, g, m1) : load_meta(pr.prob[pm.p], pm, g);
-        }
-        uint32_t nfvA = 0, nfvB = 0;
-        if (i + 1 < nb) {
-            Pos pn = pc;
-            advance(pn, pr);  // the position of block i + 1
-            const Problem &mn = pr.prob[pn.p];
-            nfvA = first_escape(mn, m1.loA, m1.hiA);
-            nfvB = first_escape(mn, m1.loB, m1.hiB);
         }
         if (pc.grp != cur.grp || pc.p != cur.p) {
             finish_group(pr, sum_halves(acc), cur, u, ub0, ub1, G0, lane);
@@ -537,17 +522,17 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_tma_kernel(const __grid_c
             decode16(rA0, make_uint2(cA.x, cA.y), B4A, wa);
             decode16(rB0, make_uint2(cB.x, cB.y), B4B, wb);
             if (eA.has & 1u)
-                fix_chunk(wa, rA0, make_uint2(cA.x, cA.y), m0.baseA, eA.s0, eA.limit, m0.loA, fvA, mp.esc, pr.err, scr);
+                fix_chunk(wa, rA0, make_uint2(cA.x, cA.y), m0.baseA, eA.s0, eA.limit, mp.esc, pr.err, scr);
             if (eB.has & 1u)
-                fix_chunk(wb, rB0, make_uint2(cB.x, cB.y), m0.baseB, eB.s0, eB.limit, m0.loB, fvB, mp.esc, pr.err, scr);
+                fix_chunk(wb, rB0, make_uint2(cB.x, cB.y), m0.baseB, eB.s0, eB.limit, mp.esc, pr.err, scr);
             half_mma(acc[0], wa, wb, xw);
             load_x(xw, xl, pc.j, 1);
             decode16(rA1, make_uint2(cA.z, cA.w), B4A, wa);
             decode16(rB1, make_uint2(cB.z, cB.w), B4B, wb);
             if (eA.has & 2u)
-                fix_chunk(wa, rA1, make_uint2(cA.z, cA.w), m0.baseA, eA.s1, eA.limit, m0.loA, fvA, mp.esc, pr.err, scr);
+                fix_chunk(wa, rA1, make_uint2(cA.z, cA.w), m0.baseA, eA.s1, eA.limit, mp.esc, pr.err, scr);
             if (eB.has & 2u)
-                fix_chunk(wb, rB1, make_uint2(cB.z, cB.w), m0.baseB, eB.s1, eB.limit, m0.loB, fvB, mp.esc, pr.err, scr);
+                fix_chunk(wb, rB1, make_uint2(cB.z, cB.w), m0.baseB, eB.s1, eB.limit, mp.esc, pr.err, scr);
             half_mma(acc[1], wa, wb, xw);
         }
         if (i + S < nb) advance(pi, pr);
@@ -555,8 +540,6 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_tma_kernel(const __grid_c
         advance(pc, pr);
         m0 = m1;
         m1 = m2;
-        fvA = nfvA;
-        fvB = nfvB;
         if (++s == S) {
             s = 0;
             parity ^= 1u;
