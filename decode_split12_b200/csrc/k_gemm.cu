@@ -265,17 +265,12 @@ __device__ __forceinline__ Layout layout(uint32_t sb, const Params<NP> &p) {
 // the chunk) from the stage into the A buffer, patching escapes.  Called by
 // whole quads (the four lanes of a quad share the row).
 // Per-tile metadata of one row: base and escape offsets.
+// (Escape values are read when a unit needs them: fetching a row's first
+// two one unit ahead cost more per unit than it hid, 6 % at M = 16.)
 struct RowMeta {
     uint32_t base, lo, hi;
-    uint32_t fv0, fv1;  // the tile row's first two escape values (fetched one unit ahead)
-    int pi;             // the matrix the unit belongs to
+    int pi;  // the matrix the unit belongs to
 };
-
-__device__ __forceinline__ void fetch_escapes(const Problem &p, RowMeta &m) {
-    m.fv0 = m.fv1 = 0;
-    if (m.lo < m.hi && m.lo < p.n_esc) m.fv0 = __ldg(p.esc + m.lo);
-    if (m.lo + 1 < m.hi && m.lo + 1 < p.n_esc) m.fv1 = __ldg(p.esc + m.lo + 1);
-}
 
 // Rows past the end (zeros from the copy engine) read the last row's
 // metadata but report no escapes.
@@ -323,7 +318,6 @@ __device__ __forceinline__ RowMeta load_row_meta(const Params<NP> &P, UPos q, in
     m.lo = __ldg(p.esc_off + t);
     m.hi = __ldg(p.esc_off + t + 1);
     if (n >= p.N) m.hi = m.lo;
-    m.fv0 = m.fv1 = 0;
     m.pi = q.p;
     return m;
 }
@@ -394,8 +388,7 @@ __device__ __forceinline__ void decode_row(const Problem &p, uint32_t *err, uint
                 mm &= mm - 1;
                 uint16_t v = 0;
                 if (idx < limit)
-                    v = idx == lo ? static_cast<uint16_t>(rm.fv0)
-                                  : (idx == lo + 1 ? static_cast<uint16_t>(rm.fv1) : __ldg(p.esc + idx));
+                    v = __ldg(p.esc + idx);
                 else
                     raise_flag(err, S12_FLAG_ESC_RANGE);
                 ++idx;
@@ -601,13 +594,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         int s = 0, a = 0;
         uint32_t round = 0, around = 0, tiles = 0;
         // the row metadata of the next two units is in flight while a unit is decoded
-        RowMeta m0 = {0, 0, 0, 0, 0, 0}, m1 = {0, 0, 0, 0, 0, 0};
+        RowMeta m0 = {0, 0, 0, 0}, m1 = {0, 0, 0, 0};
         UPos q = q0;
         UPos qm = q;  // the unit whose metadata is loaded next
-        if (u0 < u1) {
-            m0 = load_row_meta(p, qm, r);
-            fetch_escapes(p.prob[m0.pi], m0);
-        }
+        if (u0 < u1) m0 = load_row_meta(p, qm, r);
         next(qm, p);
         if (u0 + 1 < u1) m1 = load_row_meta(p, qm, r);
         next(qm, p);
@@ -620,7 +610,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                 m2 = load_row_meta(p, qm, r);
                 next(qm, p);
             }
-            if (u + 1 < u1) fetch_escapes(p.prob[m1.pi], m1);  // m1's offsets arrived during the previous unit
             const bool w = bar_wait(L.full + 8 * s, round & 1u) && bar_wait(L.a_empty + 8 * a, (around & 1u) ^ 1u);
             if (!__all_sync(0xFFFFFFFFu, w)) {
                 raise_flag(p.err, S12_FLAG_TIMEOUT);
