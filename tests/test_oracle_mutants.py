@@ -42,6 +42,12 @@ MUTANTS = {
     "last_plane_unpadded": [("L->total = L->off_esc + pad_to_align(2 * n_esc);",
                              "L->total = L->off_esc + 2 * n_esc;")],
     "entropy_in_nats": [("h -= p * log2(p);", "h -= p * log(p);")],
+    "silu_exp_sign_flipped": [("h[i] = g[i] / (1.0 + exp(-g[i])) * u[i];",
+                               "h[i] = g[i] / (1.0 + exp(g[i])) * u[i];")],
+    "silu_applied_to_up": [("h[i] = g[i] / (1.0 + exp(-g[i])) * u[i];",
+                            "h[i] = u[i] / (1.0 + exp(-u[i])) * g[i];")],
+    "sigmoid_instead_of_silu": [("h[i] = g[i] / (1.0 + exp(-g[i])) * u[i];",
+                                 "h[i] = 1.0 / (1.0 + exp(-g[i])) * u[i];")],
     "escape_stored_byte_swapped": [("esc[2 * written] = (uint8_t)(v & 0xFF);\n                esc[2 * written + 1] = (uint8_t)(v >> 8);",
                                     "esc[2 * written] = (uint8_t)(v >> 8);\n                esc[2 * written + 1] = (uint8_t)(v & 0xFF);")],
 }
@@ -83,6 +89,11 @@ def _battery(o: Oracle):
     bi = o.encode(wl.to_bf16_bits(vals))
     y, s = o.gemv_f64(bi, np.full((1, 256), 0x3F80, np.uint16))
     assert np.array_equal(y[0], vals.sum(1)) and np.array_equal(s[0], np.abs(vals).sum(1))
+    # gated-MLP activation: textbook values of t * logistic(t)
+    e = np.e
+    h = o.silu_mul_f64(np.array([1.0, 2.0, 64.0, -64.0, 0.0]), np.array([2.0, 1.0, 3.0, 3.0, 5.0]))
+    assert abs(h[0] - 2 * e / (1 + e)) < 1e-14 and abs(h[1] - 2 * e * e / (1 + e * e)) < 1e-14
+    assert abs(h[2] - 192.0) < 1e-10 and abs(h[3]) < 1e-20 and h[4] == 0.0
     # entropy near the pages' ~2.6 bits
     st = o.stats(o.encode(wl.normal_with_outliers(64, 2048, 0.02, 0.0, 0)))
     assert 2.4 <= st["exp_entropy_bits"] <= 2.8
