@@ -48,8 +48,16 @@ MUTANTS = {
                             "h[i] = u[i] / (1.0 + exp(-u[i])) * g[i];")],
     "sigmoid_instead_of_silu": [("h[i] = g[i] / (1.0 + exp(-g[i])) * u[i];",
                                  "h[i] = 1.0 / (1.0 + exp(-g[i])) * u[i];")],
-    "escape_stored_byte_swapped": [("esc[2 * written] = (uint8_t)(v & 0xFF);\n                esc[2 * written + 1] = (uint8_t)(v >> 8);",
-                                    "esc[2 * written] = (uint8_t)(v >> 8);\n                esc[2 * written + 1] = (uint8_t)(v & 0xFF);")],
+    "v2_count_check_dropped": [("            if (seen != count) return ORACLE_ERR_CORRUPT;\n", "")],
+    "v2_row_offset_ignored": [("        uint64_t k = lo; /* next escape of this row */",
+                               "        uint64_t k = 0; /* next escape of this row */")],
+    "v2_base_and_count_bytes_swapped": [
+        ("        tmeta[2 * t] = (uint8_t)b;\n        tmeta[2 * t + 1] = (uint8_t)count;",
+         "        tmeta[2 * t + 1] = (uint8_t)b;\n        tmeta[2 * t] = (uint8_t)count;"),
+        ("uint32_t b = tmeta[2 * t], count = tmeta[2 * t + 1], seen = 0;",
+         "uint32_t b = tmeta[2 * t + 1], count = tmeta[2 * t], seen = 0;")],
+    "escape_stored_byte_swapped": [("esc[2 * *written] = (uint8_t)(v & 0xFF);\n            esc[2 * *written + 1] = (uint8_t)(v >> 8);",
+                                    "esc[2 * *written] = (uint8_t)(v >> 8);\n            esc[2 * *written + 1] = (uint8_t)(v & 0xFF);")],
 }
 
 
@@ -89,6 +97,21 @@ def _battery(o: Oracle):
     bi = o.encode(wl.to_bf16_bits(vals))
     y, s = o.gemv_f64(bi, np.full((1, 256), 0x3F80, np.uint16))
     assert np.array_equal(y[0], vals.sum(1)) and np.array_equal(s[0], np.abs(vals).sum(1))
+    # container version 2: round trip, agreement with version 1's metadata,
+    # a corrupted tile count refused
+    wv = allp[wl.rng_for(0, 1).permutation(allp.size)].reshape(512, 128)
+    assert np.array_equal(o.decode_v2(o.encode_v2(wv)), wv)
+    w2, _ = wl.escape_stress(0.05, seed=2, rows=16, cols=1024)
+    b1, b2 = o.encode(w2), o.encode_v2(w2)
+    n_t = 16 * 1024 // 128
+    off_t = 256 + 16 * 1024 + 8192        # both versions: header, raw, code planes first
+    assert np.array_equal(b2[off_t:off_t + 2 * n_t:2], b1[off_t:off_t + n_t])
+    e1 = b1[off_t + 256:off_t + 256 + 4 * (n_t + 1)].view(np.uint32)
+    assert np.array_equal(b2[off_t + 1:off_t + 2 * n_t:2].astype(np.uint32), np.diff(e1))
+    k = int(np.flatnonzero(b2[off_t + 1:off_t + 2 * n_t:2])[0])
+    bad = b2.copy()
+    bad[off_t + 2 * k + 1] += 1
+    assert o.decode_v2_rc(bad) != 0
     # gated-MLP activation: textbook values of t * logistic(t)
     e = np.e
     h = o.silu_mul_f64(np.array([1.0, 2.0, 64.0, -64.0, 0.0]), np.array([2.0, 1.0, 3.0, 3.0, 5.0]))
