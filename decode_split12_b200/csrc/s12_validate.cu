@@ -130,3 +130,116 @@ extern "C" int s12_plane_hashes_host(const void *container, size_t bytes, uint64
     out[4] = fnv1a64(c + g.off_esc, 2 * g.n_esc);
     return S12_OK;
 }
+
+// ---------------------------------------------------------------------------
+// Container version 2 (a compact tile header) as a storage format.  Same
+// raw, code and escape planes; per tile one u16 = base | escape count << 8
+// and per row one u32 escape offset, instead of a u8 base and a u32 offset
+// per tile: 2 bytes per tile + 4 per row instead of 5 per tile, toward the
+// 24.967 % payload reduction of "Lossless LLM Weight Compression vs 8-bit
+// GGUF" (English edition, opening summary).  The kernels read version 1;
+// these calls convert in host memory, for storage or transfer.
+
+namespace s12 {
+namespace {
+
+struct Geometry2 {
+    uint64_t rows, cols, n_tiles, n_esc;
+    uint64_t off_raw, off_code, off_tmeta, off_row_esc, off_esc, total;
+};
+
+Geometry2 geometry2(uint64_t rows, uint64_t cols, uint64_t n_esc) {
+    Geometry2 g;
+    g.rows = rows;
+    g.cols = cols;
+    g.n_tiles = rows * (cols / kTile);
+    g.n_esc = n_esc;
+    g.off_raw = kHeaderBytes;
+    g.off_code = g.off_raw + align_up(rows * cols, kAlign);
+    g.off_tmeta = g.off_code + align_up(rows * cols / 2, kAlign);
+    g.off_row_esc = g.off_tmeta + align_up(2 * g.n_tiles, kAlign);
+    g.off_esc = g.off_row_esc + align_up(4 * (rows + 1), kAlign);
+    g.total = g.off_esc + align_up(2 * n_esc, kAlign);
+    return g;
+}
+
+void wr32(uint8_t *p, uint32_t v) {
+    for (int i = 0; i < 4; ++i) p[i] = static_cast<uint8_t>(v >> (8 * i));
+}
+
+}  // namespace
+}  // namespace s12
+
+extern "C" int s12_to_v2_host(const void *v1, size_t v1_bytes, void *dst, size_t dst_cap, size_t *bytes_out) {
+    if (!v1 || !bytes_out) return S12_ERR_ARG;
+    s12_report rep;
+    const int rc = s12_validate_host(v1, v1_bytes, &rep);
+    if (rc != S12_OK) return rc;
+    const uint8_t *c = static_cast<const uint8_t *>(v1);
+    const Geometry g = geometry(rd64(c + 8), rd64(c + 16), rd64(c + 32));
+    const Geometry2 g2 = geometry2(g.rows, g.cols, g.n_esc);
+    *bytes_out = g2.total;
+    if (!dst) return S12_OK;
+    if (dst_cap < g2.total) return S12_ERR_CAPACITY;
+    uint8_t *d = static_cast<uint8_t *>(dst);
+    std::memset(d, 0, g2.total);
+    std::memcpy(d, c, 64);
+    wr32(d + 4, 2);
+    std::memcpy(d + g2.off_raw, c + g.off_raw, g.rows * g.cols);
+    std::memcpy(d + g2.off_code, c + g.off_code, g.rows * g.cols / 2);
+    std::memcpy(d + g2.off_esc, c + g.off_esc, 2 * g.n_esc);
+    const uint8_t *off = c + g.off_esc_off;
+    const uint64_t T = g.cols / kTile;
+    for (uint64_t t = 0; t < g.n_tiles; ++t) {
+        const uint32_t count = rd32(off + 4 * (t + 1)) - rd32(off + 4 * t);  // <= 128 in a valid container
+        d[g2.off_tmeta + 2 * t] = c[g.off_base + t];
+        d[g2.off_tmeta + 2 * t + 1] = static_cast<uint8_t>(count);
+    }
+    for (uint64_t r = 0; r <= g.rows; ++r) wr32(d + g2.off_row_esc + 4 * r, rd32(off + 4 * (r * T)));
+    return S12_OK;
+}
+
+extern "C" int s12_from_v2_host(const void *v2, size_t v2_bytes, void *dst, size_t dst_cap, size_t *bytes_out) {
+    if (!v2 || !bytes_out) return S12_ERR_ARG;
+    const uint8_t *c = static_cast<const uint8_t *>(v2);
+    if (v2_bytes < kHeaderBytes || std::memcmp(c, "S12\0", 4) != 0 || rd32(c + 4) != 2 ||
+        rd32(c + 24) != static_cast<uint32_t>(kTile) || rd32(c + 28) != 0)
+        return S12_ERR_CORRUPT;
+    for (int i = 40; i < 64; ++i)
+        if (c[i]) return S12_ERR_CORRUPT;
+    const uint64_t rows = rd64(c + 8), cols = rd64(c + 16), n_esc = rd64(c + 32);
+    if (rows == 0 || cols == 0 || cols % kTile || rows >= (uint64_t(1) << 32) || cols >= (uint64_t(1) << 32) ||
+        rows * cols >= (uint64_t(1) << 32) || n_esc > rows * cols)
+        return S12_ERR_CORRUPT;
+    const Geometry2 g2 = geometry2(rows, cols, n_esc);
+    if (g2.total > v2_bytes) return S12_ERR_CORRUPT;
+    const Geometry g = geometry(rows, cols, n_esc);
+    // the row offsets and tile counts must describe the escape stream exactly
+    const uint8_t *row_esc = c + g2.off_row_esc, *tmeta = c + g2.off_tmeta;
+    const uint64_t T = cols / kTile;
+    if (rd32(row_esc) != 0 || rd32(row_esc + 4 * rows) != n_esc) return S12_ERR_CORRUPT;
+    for (uint64_t r = 0; r < rows; ++r) {
+        uint64_t k = rd32(row_esc + 4 * r);
+        for (uint64_t j = 0; j < T; ++j) k += tmeta[2 * (r * T + j) + 1];
+        if (k != rd32(row_esc + 4 * (r + 1))) return S12_ERR_CORRUPT;
+    }
+    *bytes_out = g.total;
+    if (!dst) return S12_OK;
+    if (dst_cap < g.total) return S12_ERR_CAPACITY;
+    uint8_t *d = static_cast<uint8_t *>(dst);
+    std::memset(d, 0, g.total);
+    std::memcpy(d, c, 64);
+    wr32(d + 4, 1);
+    std::memcpy(d + g.off_raw, c + g2.off_raw, rows * cols);
+    std::memcpy(d + g.off_code, c + g2.off_code, rows * cols / 2);
+    std::memcpy(d + g.off_esc, c + g2.off_esc, 2 * n_esc);
+    uint64_t k = 0;
+    for (uint64_t t = 0; t < g.n_tiles; ++t) {
+        if (t % T == 0) k = rd32(row_esc + 4 * (t / T));
+        d[g.off_base + t] = tmeta[2 * t];
+        wr32(d + g.off_esc_off + 4 * t, static_cast<uint32_t>(k));
+        k += tmeta[2 * t + 1];
+    }
+    wr32(d + g.off_esc_off + 4 * g.n_tiles, static_cast<uint32_t>(n_esc));
+    return S12_OK;
+}

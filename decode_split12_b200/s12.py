@@ -37,7 +37,8 @@ EXPORTED = (
     "s12_error_string", "s12_device_check", "s12_container_bytes", "s12_encode_ws_bytes", "s12_encode",
     "s12_open", "s12_decode", "s12_gemv_ws_bytes", "s12_gemv", "s12_gemv_multi_ws_bytes", "s12_gemv_multi",
     "s12_gemv_noalloc", "s12_gemv_swiglu", "s12_gemm_ws_bytes", "s12_gemm_skinny", "s12_gemm_multi_ws_bytes",
-    "s12_gemm_skinny_multi", "s12_validate_host", "s12_plane_hashes_host", "s12_fnv1a64", "s12_stats_ws_bytes",
+    "s12_gemm_skinny_multi", "s12_validate_host", "s12_plane_hashes_host", "s12_fnv1a64",
+    "s12_to_v2_host", "s12_from_v2_host", "s12_stats_ws_bytes",
     "s12_stats", "s12_bf16_gemv",
 )
 
@@ -114,6 +115,9 @@ def _lib() -> C.CDLL:
         lib.s12_validate_host.restype = C.c_int
         lib.s12_plane_hashes_host.argtypes = [_P, _SZ, C.POINTER(C.c_uint64)]
         lib.s12_plane_hashes_host.restype = C.c_int
+        for fn in ("s12_to_v2_host", "s12_from_v2_host"):
+            getattr(lib, fn).argtypes = [_P, _SZ, _P, _SZ, C.POINTER(_SZ)]
+            getattr(lib, fn).restype = C.c_int
         lib.s12_fnv1a64.argtypes = [_P, _SZ]
         lib.s12_fnv1a64.restype = C.c_uint64
         lib.s12_gemm_multi_ws_bytes.argtypes = [C.POINTER(View), C.c_int, C.POINTER(C.c_int)]
@@ -422,3 +426,23 @@ def s12_plane_hashes_host(container):
 def s12_fnv1a64(data: bytes) -> int:
     buf = C.create_string_buffer(bytes(data), len(data))
     return int(_lib().s12_fnv1a64(C.cast(buf, C.c_void_p), len(data)))
+
+
+def _convert(fn_name: str, container) -> np.ndarray:
+    b = _host_bytes(container)
+    fn = getattr(_lib(), fn_name)
+    n = _SZ(0)
+    _check(fn(b.ctypes.data_as(C.c_void_p), b.size, None, 0, C.byref(n)), fn_name)
+    out = np.zeros(n.value, np.uint8)
+    _check(fn(b.ctypes.data_as(C.c_void_p), b.size, out.ctypes.data_as(C.c_void_p), out.size, C.byref(n)), fn_name)
+    return out
+
+
+def to_v2_host(container) -> np.ndarray:
+    """A version 1 container (host array or tensor) as the compact version 2."""
+    return _convert("s12_to_v2_host", container)
+
+
+def from_v2_host(container) -> np.ndarray:
+    """A version 2 container back to version 1 (what the kernels read)."""
+    return _convert("s12_from_v2_host", container)

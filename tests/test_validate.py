@@ -137,3 +137,44 @@ def test_structure_free_bytes_caught_by_hashes(oracle, blob):
     assert rc == s12.S12_OK and rep["notes"] == 1
     rc, rep = _corrupt_and_judge(oracle, b, lambda c: c.__setitem__(100, 1))   # header padding
     assert rc == s12.S12_OK and rep["notes"] == 1
+
+
+@pytest.mark.parametrize("shape,kind", [((1, 128), "normal"), ((37, 640), "normal"), ((64, 1024), "stress"),
+                                        ((16, 4096), "student")])
+def test_v2_conversion_matches_oracle_and_round_trips(oracle, shape, kind):
+    """The library's host conversion to container version 2 equals the
+    oracle's version 2 encoder byte for byte, and converting back gives the
+    version 1 container byte for byte."""
+    r, c = shape
+    if kind == "stress":
+        w, _ = wl.escape_stress(0.02, 1, r, c)
+    elif kind == "student":
+        w = wl.student_t_scaled(r, c, 2)
+    else:
+        w = wl.normal_with_outliers(r, c, 0.02, 0.01, r + c)
+    v1 = oracle.encode(w)
+    v2 = s12.to_v2_host(v1)
+    assert np.array_equal(v2, oracle.encode_v2(w))
+    assert v2.size <= v1.size
+    assert np.array_equal(s12.from_v2_host(v2), v1)
+
+
+def test_v2_conversion_refuses_corrupt_sources(oracle):
+    w, _ = wl.escape_stress(0.05, 4, 16, 1024)
+    v1 = oracle.encode(w)
+    bad = v1.copy()
+    bad[1] = ord("X")
+    with pytest.raises(s12.S12Error):
+        s12.to_v2_host(bad)
+    v2 = oracle.encode_v2(w)
+    n_esc = int(v2[32:40].view(np.uint64)[0])
+    n_t = 16 * 1024 // 128
+    off_t = 256 + 16 * 1024 + 8192
+    k = int(np.flatnonzero(v2[off_t + 1:off_t + 2 * n_t:2])[0])
+    bad2 = v2.copy()
+    bad2[off_t + 2 * k + 1] += 1            # a tile count that no longer adds up to its row's span
+    with pytest.raises(s12.S12Error):
+        s12.from_v2_host(bad2)
+    with pytest.raises(s12.S12Error):
+        s12.from_v2_host(v1)                # a version 1 container is not version 2
+    assert n_esc > 0
