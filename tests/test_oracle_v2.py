@@ -6,6 +6,7 @@ counts, per-row offsets), the closed-form size, and corruption checks."""
 import numpy as np
 import pytest
 
+from conftest import golden_expected_bytes, golden_two_tiles_weights, load_golden
 from decode_split12_b200 import workloads as wl
 
 ALIGN = 256
@@ -112,3 +113,18 @@ def test_v2_corruptions_detected(oracle):
     assert bad(lambda c: c.__setitem__(4, 1))                                               # version 1 header
     # a version 1 container is not a version 2 one
     assert oracle.decode_v2_rc(oracle.encode(w)) != 0
+
+
+def test_v2_golden_two_tiles_bytes(oracle):
+    """The hand-derived version 2 container of the two-tile golden tensor
+    (tests/golden/two_tiles_v2.json: the version 1 golden bytes with the
+    version field and the two tile headers changed)."""
+    g1 = load_golden("two_tiles.json")
+    g2 = load_golden("two_tiles_v2.json")
+    expect = golden_expected_bytes(g1)
+    for off, hexs in g2["patch"]:
+        chunk = np.frombuffer(bytes.fromhex(hexs), np.uint8)
+        expect[off:off + chunk.size] = chunk
+    w = golden_two_tiles_weights(g1)
+    assert np.array_equal(oracle.encode_v2(w), expect)
+    assert np.array_equal(oracle.decode_v2(expect), w)

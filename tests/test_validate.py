@@ -178,3 +178,17 @@ def test_v2_conversion_refuses_corrupt_sources(oracle):
     with pytest.raises(s12.S12Error):
         s12.from_v2_host(v1)                # a version 1 container is not version 2
     assert n_esc > 0
+
+
+def test_v2_conversion_of_the_golden_container():
+    """The library's conversion of the hand-derived version 1 golden
+    container gives the hand-derived version 2 bytes, and back."""
+    from conftest import golden_expected_bytes, load_golden
+    g1, g2 = load_golden("two_tiles.json"), load_golden("two_tiles_v2.json")
+    v1 = golden_expected_bytes(g1)
+    v2 = v1.copy()
+    for off, hexs in g2["patch"]:
+        chunk = np.frombuffer(bytes.fromhex(hexs), np.uint8)
+        v2[off:off + chunk.size] = chunk
+    assert np.array_equal(s12.to_v2_host(v1), v2)
+    assert np.array_equal(s12.from_v2_host(v2), v1)
