@@ -29,6 +29,11 @@
 //               core reads; then, at the end of each tile, the epilogue:
 //               tcgen05.ld of the accumulators and the stores of Y.
 //
+// A call may hold up to S12_GEMM_MAX_PROBLEMS matrices (s12_gemm_skinny_multi,
+// for instance the experts of a mixture-of-experts block), each with its own
+// shape, token rows and output; they share the tensor core's N (the largest
+// M rounded up to 16), and their units are numbered matrix after matrix.
+//
 // Work split (stream-K): the (tile, tile column) units are dealt to the CTAs in
 // equal contiguous ranges.  A tile covered whole by one CTA goes straight to
 // Y; a tile shared by several CTAs is finished by the last of them to
