@@ -50,7 +50,13 @@
  *     OR into it S12_FLAG_* bits when they meet corrupt data.  They never
  *     trap or hang: the offending escape index is clamped and work goes on.
  *     The caller reads the word back (and clears it) when it wants to.
- *   - The library keeps no mutable global state and is thread-safe.
+ *   - Global state: per-device caches filled once and then only read (the
+ *     SM count, the tensor-map encoder's entry point, the static workspace's
+ *     device address) and ONE mutable object, the static workspace of
+ *     s12_gemv_noalloc (documented there).  Every other call keeps no
+ *     state between calls, and all calls are thread-safe.
+ *   - Citations: every entry point names the page and section it follows,
+ *     in a "Follows:" line, or says that the pages have no counterpart.
  */
 #ifndef S12_H
 #define S12_H
@@ -123,7 +129,9 @@ const char *s12_error_string(int status);
 int s12_device_check(void);
 
 /* Container size in bytes for a shape and escape count (closed form of the
- * layout above); 0 when the shape is invalid (cols % 128 != 0 or zero). */
+ * layout above); 0 when the shape is invalid (cols % 128 != 0 or zero).
+ * Follows: [T] key points (a fixed 12-bit rate: 1.5 bytes per weight, plus
+ * the tile headers and escapes of this container). */
 uint64_t s12_container_bytes(int64_t rows, int64_t cols, uint64_t n_esc);
 
 /* ---- encoder ([W] "What did the GLM-5.2 experiment actually prove?":
@@ -134,7 +142,10 @@ uint64_t s12_container_bytes(int64_t rows, int64_t cols, uint64_t n_esc);
  * content, 16-byte aligned, owned by the caller). */
 size_t s12_encode_ws_bytes(int64_t rows, int64_t cols);
 
-/* Encode a row-major BF16 matrix `w` (device, rows x cols, cols % 128 == 0,
+/* Follows: [W] "What did the GLM-5.2 experiment actually prove?" (short
+ * fixed codes, an exact escape stream); [T] technical deep dive (128-weight
+ * blocks sharing a base).
+ * Encode a row-major BF16 matrix `w` (device, rows x cols, cols % 128 == 0,
  * rows*cols < 2^32) into a Split12 container.
  *   dst == NULL: only computes *bytes_out (the exact container size).
  *   dst != NULL: writes the whole container (header, planes, zero padding)
@@ -147,7 +158,9 @@ size_t s12_encode_ws_bytes(int64_t rows, int64_t cols);
 int s12_encode(const uint16_t *w, int64_t rows, int64_t cols, void *dst, size_t dst_cap,
                size_t *bytes_out, void *ws, size_t ws_bytes, void *stream);
 
-/* Validate the 64-byte header of a container (device, `bytes` long) and
+/* Follows: the container layout above, which restates [M] section 1 (the
+ * BF16 bit fields) and [T] key points (tile base, escape stream).
+ * Validate the 64-byte header of a container (device, `bytes` long) and
  * fill *out with its shape and plane pointers.  Copies the header to the
  * host and so SYNCHRONISES (the legacy default stream).  S12_ERR_CORRUPT on
  * a bad magic, version, tile size, flags, shape or a size above `bytes`. */
@@ -156,7 +169,10 @@ int s12_open(const void *container, size_t bytes, s12_view *out);
 /* ---- standalone decode ([T] key points: one integer ADD per weight,
  * code 15 read from the escape stream) ---- */
 
-/* Decode the whole container to BF16 `out` (device, rows x cols, row-major).
+/* Follows: [T] key points (exponent = base + code, one integer ADD; code
+ * 15 read from the separate escape stream); [W] "What does 'lossless' mean
+ * for LLM weights?" (the exact round trip is the definition).
+ * Decode the whole container to BF16 `out` (device, rows x cols, row-major).
  * Bit-exact: out equals the encoded matrix. */
 int s12_decode(const s12_view *v, uint16_t *out, uint32_t *err_flag, void *stream);
 
@@ -170,7 +186,9 @@ int s12_decode(const s12_view *v, uint16_t *out, uint32_t *err_flag, void *strea
  * size serves every matrix of a model on that device. */
 size_t s12_gemv_ws_bytes(const s12_view *v, int B);
 
-/* y[b][n] = sum_k W[n][k] * x[b][k] for b < B, 1 <= B <= 8.
+/* Follows: [W] "What does 'lossless' mean for LLM weights?" (decode into
+ * registers and multiply at once); [T] key points (one-ADD decode).
+ * y[b][n] = sum_k W[n][k] * x[b][k] for b < B, 1 <= B <= 8.
  *   x:  device BF16, B x cols row-major.
  *   y:  device FP32, B x rows row-major (4-byte alignment suffices),
  *       overwritten.
@@ -197,7 +215,8 @@ int s12_gemv(const s12_view *v, const uint16_t *x, int B, float *y, void *ws, si
  * and the SM count, not on B. */
 size_t s12_gemv_multi_ws_bytes(const s12_view *views, int count, int B);
 
-/* Up to S12_GEMV_MAX_PROBLEMS independent fused decode-GEMVs in ONE kernel
+/* Follows: as s12_gemv ([W] "What does 'lossless' mean for LLM weights?").
+ * Up to S12_GEMV_MAX_PROBLEMS independent fused decode-GEMVs in ONE kernel
  * launch: for i < count, y[i][b][n] = sum_k W_i[n][k] * x[i][b][k], b < B.
  *   views: host array of `count` opened containers (shapes may differ).
  *   x, y:  host arrays of `count` device pointers, laid out as in s12_gemv.
@@ -213,7 +232,10 @@ size_t s12_gemv_multi_ws_bytes(const s12_view *views, int count, int B);
 int s12_gemv_multi(const s12_view *views, int count, const uint16_t *const *x, int B, float *const *y,
                    void *ws, size_t ws_bytes, uint32_t *err_flag, void *stream);
 
-/* Fused decode-GEMV with a SwiGLU epilogue, for a gated MLP's gate and up
+/* Follows: [W] "What does 'lossless' mean for LLM weights?" (decoded
+ * weights used at once by the decode kernel; the gated-MLP epilogue is this
+ * library's own addition).
+ * Fused decode-GEMV with a SwiGLU epilogue, for a gated MLP's gate and up
  * projections (F rows each): h[b][f] = silu(g[b][f]) * u[b][f], where
  * g = W_gate x_b, u = W_up x_b and silu(t) = t / (1 + exp(-t)), rounded to
  * BF16 (round to nearest even).
@@ -234,8 +256,9 @@ int s12_gemv_multi(const s12_view *views, int count, const uint16_t *const *x, i
 int s12_gemv_swiglu(const s12_view *v, const uint16_t *x, int B, uint16_t *h, void *ws, size_t ws_bytes,
                     uint32_t *err_flag, void *stream);
 
-/* s12_gemv for callers that cannot allocate device memory (no counterpart
- * in the pages: it exists for integration, not for the method).  Examples are
+/* The pages have no counterpart of this call: it exists for integration,
+ * not for the method.
+ * s12_gemv for callers that cannot allocate device memory.  Examples are
  * a plugin whose host engine owns all device memory through its own
  * allocator, code under a fixed memory budget, or a path where cudaMalloc's
  * implicit synchronisation is not allowed.  Same arguments and result as
@@ -261,7 +284,11 @@ int s12_gemv_noalloc(const s12_view *v, const uint16_t *x, int B, float *y, uint
 /* Workspace bytes s12_gemm_skinny needs for this container and M. */
 size_t s12_gemm_ws_bytes(const s12_view *v, int M);
 
-/* y[m][n] = sum_k W[n][k] * x[m][k] for 16 <= M <= 256.
+/* Follows: [W] "How does this compare with prior lossless systems?" (a
+ * fused decompression-GEMM: the weights are decoded inside the matrix
+ * product, not to a BF16 copy in memory); [T] key points (the one-ADD
+ * decode feeding tensor-core kernels).
+ * y[m][n] = sum_k W[n][k] * x[m][k] for 16 <= M <= 256.
  *   x: device BF16, M x cols row-major.  y: device FP32, M x rows row-major,
  *   overwritten.  ws: device scratch of s12_gemm_ws_bytes(v, M) bytes,
  *   ZERO-FILLED before its first use; every call leaves it zero-filled.
@@ -274,7 +301,9 @@ int s12_gemm_skinny(const s12_view *v, const uint16_t *x, int M, float *y, void 
  * with token rows M[i] (0 for invalid arguments). */
 size_t s12_gemm_multi_ws_bytes(const s12_view *views, int count, const int *M);
 
-/* Up to S12_GEMM_MAX_PROBLEMS independent fused decode-skinny-GEMMs in ONE
+/* Follows: as s12_gemm_skinny ([W] "How does this compare with prior
+ * lossless systems?": fused decompression-GEMM; [T] key points).
+ * Up to S12_GEMM_MAX_PROBLEMS independent fused decode-skinny-GEMMs in ONE
  * kernel launch: for i < count, y[i][m][n] = sum_k W_i[n][k] * x[i][m][k]
  * for m < M[i], 1 <= M[i] <= 256 (below 16 too: every matrix is multiplied
  * at the call's shared padded M).  Built for a mixture-of-experts block,
@@ -303,7 +332,9 @@ int s12_gemm_skinny_multi(const s12_view *views, int count, const uint16_t *cons
 /* Workspace bytes s12_stats needs (device scratch). */
 size_t s12_stats_ws_bytes(void);
 
-/* Fill *out with sizes, rates and the exponent histogram/entropy of the
+/* Follows: [M] section 1 entropy table (exponent entropy in bits); [T] key
+ * points (escape rate, size ratio).
+ * Fill *out with sizes, rates and the exponent histogram/entropy of the
  * decoded weights.  Runs a histogram kernel and SYNCHRONISES `stream`. */
 int s12_stats(const s12_view *v, s12_stats_t *out, void *ws, size_t ws_bytes, void *stream);
 
@@ -326,7 +357,9 @@ typedef struct s12_report {
     uint64_t n_esc_counted; /* code-15 nibbles in the tiles checked             */
 } s12_report;
 
-/* Check a whole container in HOST memory (for instance a file read before
+/* Follows: [W] "A 14-day production-readiness pilot" (verify what was
+ * loaded; inject corruption and confirm that it is detected).
+ * Check a whole container in HOST memory (for instance a file read before
  * it is copied to the device): S12_OK when it is valid, S12_ERR_CORRUPT with
  * *out describing the first problem otherwise (S12_ERR_ARG for NULLs).  A
  * valid container decodes without any err_flag bit.  Raw bytes and escape
@@ -334,17 +367,23 @@ typedef struct s12_report {
  * s12_plane_hashes_host. */
 int s12_validate_host(const void *container, size_t bytes, s12_report *out);
 
-/* 64-bit FNV-1a hashes of the exact bytes of the five planes, in the order
+/* Follows: [W] "A 14-day production-readiness pilot" (hash what was
+ * stored and compare after loading).
+ * 64-bit FNV-1a hashes of the exact bytes of the five planes, in the order
  * raw, code, base, esc_off, esc (padding excluded), of a container in HOST
  * memory with a valid header.  Any change of a single byte changes its
  * plane's hash.  Store them at encode time and compare after loading. */
 int s12_plane_hashes_host(const void *container, size_t bytes, uint64_t out[5]);
 
-/* FNV-1a 64-bit hash of `bytes` bytes (offset basis 0xcbf29ce484222325,
+/* Follows: [W] "A 14-day production-readiness pilot" (the hash behind
+ * s12_plane_hashes_host).
+ * FNV-1a 64-bit hash of `bytes` bytes (offset basis 0xcbf29ce484222325,
  * prime 0x100000001b3), the function s12_plane_hashes_host uses. */
 uint64_t s12_fnv1a64(const void *data, size_t bytes);
 
-/* Container version 2, a compact tile header, as a storage format: the same
+/* Follows: [W] English edition, opening summary (the 24.967 % payload
+ * reduction leaves little room for per-tile metadata).
+ * Container version 2, a compact tile header, as a storage format: the same
  * raw, code and escape planes, with per tile ONE u16 (base | escape count
  * << 8) and per row one u32 escape offset instead of a u8 base and a u32
  * offset per tile (2 bytes per tile + 4 per row instead of 5 per tile; [W]
@@ -361,7 +400,10 @@ int s12_from_v2_host(const void *v2, size_t v2_bytes, void *dst, size_t dst_cap,
 
 /* ---- uncompressed baseline ---- */
 
-/* Plain BF16 GEMV, the comparison point for s12_gemv: y[b][n] =
+/* Follows: the plain matrix-vector product that [W] "What does 'lossless'
+ * mean for LLM weights?" says the decoded weights must reproduce; it is the
+ * uncompressed comparison point.
+ * Plain BF16 GEMV, the comparison point for s12_gemv: y[b][n] =
  * sum_k w[n][k] * x[b][k], w device BF16 rows x cols (cols % 8 == 0),
  * 1 <= B <= 8, y FP32 B x rows. */
 int s12_bf16_gemv(const uint16_t *w, int64_t rows, int64_t cols, const uint16_t *x, int B,

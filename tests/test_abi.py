@@ -32,6 +32,43 @@ def test_header_declares_entry_points():
         assert required in names
 
 
+HELPERS = ("s12_error_string", "s12_device_check")
+
+
+def declaration_comments():
+    """(name, the comment block right before its declaration) for every
+    function the header declares, in order."""
+    text = open(HEADER).read()
+    out = []
+    for m in re.finditer(r"\n(?:const )?[a-z_0-9]+ \*?(s12_[a-z0-9_]+)\(", text):
+        before = text[:m.start()].rstrip()
+        comment = ""
+        if before.endswith("*/"):
+            comment = before[before.rfind("/*"):]
+        elif before.endswith(";"):
+            # a declaration that shares the comment of the one before it
+            prev = before[:before.rfind("\n")].rstrip()
+            if prev.endswith("*/"):
+                comment = prev[prev.rfind("/*"):]
+        out.append((m.group(1), comment))
+    return out
+
+
+def test_every_entry_point_cites_its_passage():
+    """Every entry point except the status and device helpers and the
+    workspace-size queries names the page and section it follows (a
+    "Follows:" line citing [W], [M] or [T]) or states that the pages have no
+    counterpart."""
+    decls = declaration_comments()
+    assert {n for n, _ in decls} == set(declared_functions())
+    for name, comment in decls:
+        if name in HELPERS or name.endswith("_ws_bytes"):
+            continue
+        assert comment, f"{name} has no comment"
+        cited = "Follows:" in comment and re.search(r"\[(W|M|T)\]", comment)
+        assert cited or "no counterpart" in comment, f"{name} cites no passage"
+
+
 def test_every_declared_symbol_is_exported(lib):
     for name in declared_functions():
         assert hasattr(lib, name), f"{name} declared in s12.h but not exported"

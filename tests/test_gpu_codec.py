@@ -99,6 +99,26 @@ def test_single_tensor_full_size(s12, oracle):
     _roundtrip(s12, oracle, w)
 
 
+_FULL_SHAPES = {
+    "llama8b_kv_1024x4096": lambda: wl.llama8b_layer(0, 1, names=["k"])[0]["k"],
+    "llama8b_q_4096x4096": lambda: wl.llama8b_layer(0, 1, names=["q"])[0]["q"],
+    "llama8b_gate_14336x4096": lambda: wl.llama8b_layer(0, 1, names=["gate"])[0]["gate"],
+    "llama8b_down_4096x14336": lambda: wl.llama8b_layer(0, 1, names=["down"])[0]["down"],
+    "mlp70b_up_28672x8192": lambda: wl.mlp70b("up", 0),
+    "mlp70b_down_8192x28672": lambda: wl.mlp70b("down", 0),
+}
+
+
+@pytest.mark.parametrize("name", list(_FULL_SHAPES))
+def test_encode_full_shapes_byte_exact(s12, oracle, name):
+    """Every full-size matrix the GEMV and GEMM parity tests and the bench
+    use: the GPU encoder's container equals the oracle's byte for byte, and
+    the GPU decode gives W back bit for bit ("What does 'lossless' mean for
+    LLM weights?": the exact round trip is the definition)."""
+    w = _FULL_SHAPES[name]()
+    _roundtrip(s12, oracle, w)
+
+
 @pytest.mark.parametrize("rate", wl.ESCAPE_RATES)
 def test_escape_stress_full_size_decode(s12, oracle, rate):
     """8192 x 8192 at each escape rate: exact escape count and bit-exact

@@ -92,9 +92,9 @@ def test_gemm_70b_mlp_full_size_sampled(s12, oracle, name, M):
     w = wl.mlp70b(name, 0)
     x = wl.activations(M, w.shape[1], M)
     blob, view, y = _gemm(s12, w, x)
-    host = blob.cpu().numpy()
     rows = np.unique(np.concatenate([[0, w.shape[0] - 1], wl.rng_for(8, M).choice(w.shape[0], 46, replace=False)]))
-    yr, sr = oracle.gemv_rows_f64(host, x, rows)
+    # the reference starts from W: the oracle encodes the sampled rows itself
+    yr, sr = oracle.gemv_f64(oracle.encode(w[rows]), x)
     assert_within_tolerance(y[:, rows], yr, sr)
 
 
@@ -134,19 +134,22 @@ def test_gemm_multi_moe_experts_full_size(s12, oracle):
     rows per expert against the FP64 oracle, and the result equals the
     per-expert single calls within the tolerance."""
     Ms = [14, 15, 13, 14, 17, 20, 15, 20]
-    views, blobs, hosts, xs = [], [], [], []
+    views, blobs, refs, xs, samples = [], [], [], [], []
     for e, m in enumerate(Ms):
         w = wl.student_t_scaled(14336, 4096, 100 + e)
         blobs.append(s12.s12_encode(to_dev(w)))
         views.append(s12.s12_open(blobs[-1]))
-        hosts.append(blobs[-1].cpu().numpy())
+        rows = np.unique(np.concatenate([[0, 14335], wl.rng_for(9, e).choice(14336, 22, replace=False)]))
+        samples.append(rows)
+        # the reference starts from W: the oracle encodes the sampled rows itself
+        refs.append(oracle.encode(w[rows]))
         xs.append(wl.activations(m, 4096, 200 + e))
         del w
     ys = s12.s12_gemm_skinny_multi(views, [to_dev(x) for x in xs])
     torch.cuda.synchronize()
     for e, m in enumerate(Ms):
-        rows = np.unique(np.concatenate([[0, 14335], wl.rng_for(9, e).choice(14336, 22, replace=False)]))
-        yr, sr = oracle.gemv_rows_f64(hosts[e], xs[e], rows)
+        rows = samples[e]
+        yr, sr = oracle.gemv_f64(refs[e], xs[e])
         assert_within_tolerance(ys[e][:, rows].cpu().numpy(), yr, sr)
 
 
