@@ -464,7 +464,7 @@ def run_llama8b(args, world, rank):
     if not args.no_stack:
         extra["whole_stack"] = stack_extras(world)
     del ge
-    traffic = load_traffic("gemv_tma_kernel", f"llama8b_b{args.batch}")
+    traffic = load_traffic("gemv_kernel", f"llama8b_b{args.batch}")
     out = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -497,7 +497,7 @@ def run_llama8b(args, world, rank):
             "frac": round(achieved / hbm, 4),
             "traffic": (traffic or {}).get("dram_bytes_per_step"),
             "peak_kind": peak_kind,
-            "kernel": "gemv_tma_kernel",
+            "kernel": "gemv_kernel",
         },
         "clocks": sampler.summary(),
         "e2e": {"value": round(2 * layer.weights / e2e_t / 1e9 * world, 2), "unit": "GB/s",
@@ -881,7 +881,7 @@ def run_single(args, world, rank):
                          f"walked in order, > 3x L2"},
         "roofline": {"bound": "hbm", "achieved": round(alg / t / 1e9, 1), "peak": hbm, "unit": "GB/s",
                      "frac": round(alg / t / 1e9 / hbm, 4), "traffic": None, "peak_kind": peak_kind,
-                     "kernel": "gemv_tma_kernel"},
+                     "kernel": "gemv_kernel"},
         "clocks": sampler.summary(),
         "gpu_launches": steps,
         "extra": extra,

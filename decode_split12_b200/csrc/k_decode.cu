@@ -79,6 +79,7 @@ __global__ void __launch_bounds__(256) decode_kernel(DecodeParams p) {
 }
 
 int launch_decode(const s12_view *v, uint16_t *out, uint32_t *err, cudaStream_t stream) {
+    if (v->version != 1) return S12_ERR_ARG;
     DecodeParams p;
     p.raw = v->raw;
     p.code = v->code;

@@ -765,6 +765,8 @@ size_t gemm_ws_bytes(const s12_view *views, int count, const int *M) {
 
 int launch_gemm(const s12_view *views, int count, const uint16_t *const *x, const int *M, float *const *y, void *ws,
                 size_t ws_bytes, uint32_t *err, cudaStream_t stream) {
+    for (int i = 0; i < count; ++i)
+        if (views[i].version != 1) return S12_ERR_ARG;
     int sms = 0;
     if (device_sms(&sms) != cudaSuccess) return S12_ERR_CUDA;
     const Plan pl = plan(views, count, M, sms);

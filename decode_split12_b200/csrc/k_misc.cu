@@ -50,6 +50,7 @@ __global__ void __launch_bounds__(256) exp_hist_kernel(s12_view v, unsigned long
 }
 
 int launch_stats_hist(const s12_view *v, unsigned long long *hist, cudaStream_t stream) {
+    if (v->version != 1) return S12_ERR_ARG;
     int sms = 0;
     if (device_sms(&sms) != cudaSuccess) return S12_ERR_CUDA;
     if (cudaMemsetAsync(hist, 0, 256 * sizeof(unsigned long long), stream) != cudaSuccess) return S12_ERR_CUDA;

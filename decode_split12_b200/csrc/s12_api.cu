@@ -19,12 +19,23 @@ std::atomic<int> g_sms[kMaxDevices];
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3) == 0; }
 
+}  // namespace
+
 int check_view(const s12_view *v) {
-    if (!v || !v->container || !v->raw || !v->code || !v->base || !v->esc_off || !v->esc) return S12_ERR_ARG;
+    if (!v || !v->container || !v->raw || !v->code || !v->esc) return S12_ERR_ARG;
+    if (v->version == 1) {
+        if (!v->base || !v->esc_off) return S12_ERR_ARG;
+    } else if (v->version == 2) {
+        if (!v->tmeta || !v->row_esc) return S12_ERR_ARG;
+    } else {
+        return S12_ERR_ARG;
+    }
     if (v->rows == 0 || v->cols == 0 || v->cols % kTile) return S12_ERR_SHAPE;
     if (!aligned16(v->container)) return S12_ERR_ALIGN;
     return S12_OK;
 }
+
+namespace {
 
 uint32_t get_u32(const uint8_t *p) {
     return uint32_t(p[0]) | uint32_t(p[1]) << 8 | uint32_t(p[2]) << 16 | uint32_t(p[3]) << 24;
@@ -74,6 +85,23 @@ int make_tmap_u8_2d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t
 }
 
 namespace {
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+    std::call_once(g_encode_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode_tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode_tiled;
+}
+
+CUtensorMapSwizzle swizzle_mode(int swizzle) {
+    return swizzle == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+           : swizzle == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                           : CU_TENSOR_MAP_SWIZZLE_NONE;
+}
+
 int encode_2d(CUtensorMap *out, CUtensorMapDataType dtype, const void *base, uint64_t inner, uint64_t rows,
               uint64_t row_stride, uint32_t box_inner, uint32_t box_rows, int swizzle) {
     std::call_once(g_encode_once, [] {
@@ -97,6 +125,20 @@ int encode_2d(CUtensorMap *out, CUtensorMapDataType dtype, const void *base, uin
     return r == CUDA_SUCCESS ? S12_OK : S12_ERR_CUDA;
 }
 }  // namespace
+
+int make_tmap_u8_3d(CUtensorMap *out, const void *base, uint64_t inner, uint64_t d1, uint64_t d2, uint64_t stride1,
+                    uint64_t stride2, uint32_t box_inner, uint32_t box1, uint32_t box2, int swizzle) {
+    auto enc = encoder();
+    if (!enc) return S12_ERR_CUDA;
+    const cuuint64_t dims[3] = {inner, d1, d2};
+    const cuuint64_t strides[2] = {stride1, stride2};
+    const cuuint32_t box[3] = {box_inner, box1, box2};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(out, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_mode(swizzle), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? S12_OK : S12_ERR_CUDA;
+}
 
 }  // namespace s12
 
@@ -150,7 +192,8 @@ int s12_open(const void *container, size_t bytes, s12_view *out) {
     uint8_t h[64];
     if (cudaMemcpy(h, container, sizeof h, cudaMemcpyDeviceToHost) != cudaSuccess) return S12_ERR_CUDA;
     if (std::memcmp(h, "S12\0", 4) != 0) return S12_ERR_CORRUPT;
-    if (get_u32(h + 4) != 1 || get_u32(h + 24) != static_cast<uint32_t>(kTile) || get_u32(h + 28) != 0)
+    const uint32_t version = get_u32(h + 4);
+    if ((version != 1 && version != 2) || get_u32(h + 24) != static_cast<uint32_t>(kTile) || get_u32(h + 28) != 0)
         return S12_ERR_CORRUPT;
     for (int i = 40; i < 64; ++i)
         if (h[i]) return S12_ERR_CORRUPT;
@@ -159,20 +202,34 @@ int s12_open(const void *container, size_t bytes, s12_view *out) {
     if (rows >= (uint64_t(1) << 32) || cols >= (uint64_t(1) << 32) || rows * cols >= (uint64_t(1) << 32))
         return S12_ERR_CORRUPT;
     if (n_esc > rows * cols) return S12_ERR_CORRUPT;
-    const Geometry g = geometry(rows, cols, n_esc);
-    if (g.total > bytes) return S12_ERR_CORRUPT;
     const uint8_t *c = static_cast<const uint8_t *>(container);
+    std::memset(out, 0, sizeof *out);
     out->rows = rows;
     out->cols = cols;
-    out->n_tiles = g.n_tiles;
     out->n_esc = n_esc;
-    out->container_bytes = g.total;
     out->container = container;
-    out->raw = c + g.off_raw;
-    out->code = c + g.off_code;
-    out->base = c + g.off_base;
-    out->esc_off = reinterpret_cast<const uint32_t *>(c + g.off_esc_off);
-    out->esc = reinterpret_cast<const uint16_t *>(c + g.off_esc);
+    out->version = version;
+    if (version == 1) {
+        const Geometry g = geometry(rows, cols, n_esc);
+        if (g.total > bytes) return S12_ERR_CORRUPT;
+        out->n_tiles = g.n_tiles;
+        out->container_bytes = g.total;
+        out->raw = c + g.off_raw;
+        out->code = c + g.off_code;
+        out->base = c + g.off_base;
+        out->esc_off = reinterpret_cast<const uint32_t *>(c + g.off_esc_off);
+        out->esc = reinterpret_cast<const uint16_t *>(c + g.off_esc);
+    } else {
+        const Geometry2 g = geometry2(rows, cols, n_esc);
+        if (g.total > bytes) return S12_ERR_CORRUPT;
+        out->n_tiles = g.n_tiles;
+        out->container_bytes = g.total;
+        out->raw = c + g.off_raw;
+        out->code = c + g.off_code;
+        out->tmeta = reinterpret_cast<const uint16_t *>(c + g.off_tmeta);
+        out->row_esc = reinterpret_cast<const uint32_t *>(c + g.off_row_esc);
+        out->esc = reinterpret_cast<const uint16_t *>(c + g.off_esc);
+    }
     return S12_OK;
 }
 
@@ -193,27 +250,44 @@ size_t s12_gemv_multi_ws_bytes(const s12_view *views, int count, int B) {
     return gemv_ws_bytes(views, count);
 }
 
-namespace {
-// Checks shared by the GEMV calls (every entry, before any launch), then the
-// launch.  act[i] == 1 marks a SwiGLU entry: interleaved gate/up rows
-// (a multiple of 16) and a BF16 output of half the rows.
-int gemv_group(const s12_view *views, int count, const uint16_t *const *x, int B, void *const *y, const int *act,
-               void *ws, size_t ws_bytes, uint32_t *err_flag, void *stream) {
-    if (!views || !x || !y || !ws) return S12_ERR_ARG;
+}  // extern "C"
+
+namespace s12 {
+
+int gemv_check(const s12_view *views, int count, const uint16_t *const *x, int B, void *const *y, const int *out,
+               uint32_t *err_flag) {
+    if (!views || !x || !y) return S12_ERR_ARG;
     if (count < 1 || count > S12_GEMV_MAX_PROBLEMS || B < 1 || B > S12_GEMV_MAX_BATCH) return S12_ERR_SHAPE;
     for (int i = 0; i < count; ++i) {
-        int rc = check_view(views + i);
+        const int rc = check_view(views + i);
         if (rc != S12_OK) return rc;
         if (!x[i] || !y[i]) return S12_ERR_ARG;
         if (views[i].rows > 0x7FFFFFFFull || views[i].cols > 0x7FFFFFFFull) return S12_ERR_SHAPE;
-        const bool swiglu = act && act[i] == 1;
-        if (act && act[i] != 0 && act[i] != 1) return S12_ERR_ARG;
-        if (swiglu && views[i].rows % 16 != 0) return S12_ERR_SHAPE;
-        if (!aligned16(x[i]) || (swiglu ? (reinterpret_cast<uintptr_t>(y[i]) & 1) != 0 : !aligned4(y[i])))
-            return S12_ERR_ALIGN;
+        if (views[i].version != views[0].version) return S12_ERR_ARG;
+        const int o = out ? out[i] : kGemvOutF32;
+        if (o != kGemvOutF32 && o != kGemvOutSwiglu && o != kGemvOutBf16) return S12_ERR_ARG;
+        if (o == kGemvOutSwiglu && views[i].rows % 16 != 0) return S12_ERR_SHAPE;
+        const bool y_ok = o == kGemvOutF32 ? aligned4(y[i]) : (reinterpret_cast<uintptr_t>(y[i]) & 1) == 0;
+        if (!aligned16(x[i]) || !y_ok) return S12_ERR_ALIGN;
     }
-    if (!aligned16(ws) || (err_flag && !aligned4(err_flag))) return S12_ERR_ALIGN;
-    return launch_gemv(views, count, x, B, y, act, ws, ws_bytes, err_flag, static_cast<cudaStream_t>(stream));
+    if (err_flag && !aligned4(err_flag)) return S12_ERR_ALIGN;
+    return S12_OK;
+}
+
+}  // namespace s12
+
+extern "C" {
+
+namespace {
+// Checks shared by the GEMV calls (every entry, before any launch), then the
+// launch.  out[i] is the output kind of entry i (null: all FP32).
+int gemv_group(const s12_view *views, int count, const uint16_t *const *x, int B, void *const *y, const int *out,
+               void *ws, size_t ws_bytes, uint32_t *err_flag, void *stream) {
+    const int rc = gemv_check(views, count, x, B, y, out, err_flag);
+    if (rc != S12_OK) return rc;
+    if (!ws) return S12_ERR_ARG;
+    if (!aligned16(ws)) return S12_ERR_ALIGN;
+    return launch_gemv(views, count, x, B, y, out, ws, ws_bytes, err_flag, static_cast<cudaStream_t>(stream));
 }
 }  // namespace
 
@@ -229,8 +303,16 @@ int s12_gemv_swiglu(const s12_view *v, const uint16_t *x, int B, uint16_t *h, vo
                     uint32_t *err_flag, void *stream) {
     if (!v || !x || !h || !ws) return S12_ERR_ARG;
     void *out[1] = {h};
-    const int act[1] = {1};
-    return gemv_group(v, 1, &x, B, out, act, ws, ws_bytes, err_flag, stream);
+    const int kind[1] = {kGemvOutSwiglu};
+    return gemv_group(v, 1, &x, B, out, kind, ws, ws_bytes, err_flag, stream);
+}
+
+int s12_gemv_bf16(const s12_view *v, const uint16_t *x, int B, uint16_t *y, void *ws, size_t ws_bytes,
+                  uint32_t *err_flag, void *stream) {
+    if (!v || !x || !y || !ws) return S12_ERR_ARG;
+    void *out[1] = {y};
+    const int kind[1] = {kGemvOutBf16};
+    return gemv_group(v, 1, &x, B, out, kind, ws, ws_bytes, err_flag, stream);
 }
 
 int s12_gemv(const s12_view *v, const uint16_t *x, int B, float *y, void *ws, size_t ws_bytes, uint32_t *err_flag,

@@ -46,6 +46,30 @@ __host__ __device__ inline Geometry geometry(uint64_t rows, uint64_t cols, uint6
     return g;
 }
 
+// Plane offsets of a version 2 container (compact tile header): the raw,
+// code and escape planes as in version 1, and in place of the base and
+// offset planes one u16 per tile (base | escape count << 8) and one u32 per
+// row (escapes in the rows before it; the last entry is n_esc).
+struct Geometry2 {
+    uint64_t rows, cols, n_tiles, n_esc;
+    uint64_t off_raw, off_code, off_tmeta, off_row_esc, off_esc, total;
+};
+
+__host__ __device__ inline Geometry2 geometry2(uint64_t rows, uint64_t cols, uint64_t n_esc) {
+    Geometry2 g;
+    g.rows = rows;
+    g.cols = cols;
+    g.n_tiles = rows * (cols / kTile);
+    g.n_esc = n_esc;
+    g.off_raw = kHeaderBytes;
+    g.off_code = g.off_raw + align_up(rows * cols, kAlign);
+    g.off_tmeta = g.off_code + align_up(rows * cols / 2, kAlign);
+    g.off_row_esc = g.off_tmeta + align_up(2 * g.n_tiles, kAlign);
+    g.off_esc = g.off_row_esc + align_up(4 * (rows + 1), kAlign);
+    g.total = g.off_esc + align_up(2 * n_esc, kAlign);
+    return g;
+}
+
 // ---------------------------------------------------------------------------
 // Bounded waiting.  Every spin in these kernels gives up after about a second
 // at full clock, sets S12_FLAG_TIMEOUT and lets the caller unwind.

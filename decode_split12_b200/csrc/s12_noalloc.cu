@@ -17,6 +17,8 @@
 // library.
 #include <mutex>
 
+#include <cudaTypedefs.h>
+
 #include "s12_device.cuh"
 #include "s12_launch.h"
 
@@ -25,11 +27,12 @@ namespace {
 
 constexpr int kMaxSms = 160;
 constexpr uint64_t kMaxRows = 1ull << 20;
-constexpr int kWarpsPerSm = 16;       // warps per CTA of the GEMV kernel
-constexpr uint64_t kSlotBytes = 512;  // one stream-K partial: 32 lanes x 4 floats
-constexpr uint64_t kPartBytes = static_cast<uint64_t>(kMaxSms) * kWarpsPerSm * 2 * kSlotBytes;
-constexpr uint64_t kCntBytes = (kMaxRows / 16) * sizeof(uint32_t);
+// the same partial-sum and counter regions s12_gemv_ws_bytes sizes, for the
+// largest device and container this array serves
+constexpr uint64_t kPartBytes = gemv_part_bytes(kMaxSms);
+constexpr uint64_t kCntBytes = gemv_cnt_bytes(kMaxRows / 16);
 constexpr uint64_t kScratchBytes = kPartBytes + kCntBytes;
+static_assert(kScratchBytes == 2883584, "the documented size of the static workspace");
 
 // The workspace.  Host code must not use the name as an address (on the host
 // it names a stand-in object, not device memory); the device address comes
@@ -39,17 +42,37 @@ static __device__ __align__(256) uint8_t g_gemv_scratch[kScratchBytes];
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void *g_addr[kMaxDevices] = {};
+CUcontext g_ctx[kMaxDevices] = {};
+PFN_cuCtxGetCurrent_v4000 g_get_ctx = nullptr;
+std::once_flag g_get_ctx_once;
 
-// Device address of g_gemv_scratch on the current device, looked up once per
-// device (with that device current) and cached.
+// Device address of g_gemv_scratch for the current device, looked up with
+// that device current the first time it is needed and cached.  The cache is
+// keyed on the current context as well as the device: after cudaDeviceReset
+// (or with another context current) the module lives elsewhere, so the
+// address is looked up again.
 int scratch_address(void **out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return S12_ERR_CUDA;
+    std::call_once(g_get_ctx_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_get_ctx = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+    });
+    if (!g_get_ctx) return S12_ERR_CUDA;
+    CUcontext ctx = nullptr;
+    if (g_get_ctx(&ctx) != CUDA_SUCCESS) return S12_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_addr[dev]) {
+    if (!ctx || !g_addr[dev] || g_ctx[dev] != ctx) {
+        // (the lookup also makes the runtime's context current on this
+        // thread if no CUDA call has done so yet)
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_gemv_scratch) != cudaSuccess || !p) return S12_ERR_CUDA;
+        if (g_get_ctx(&ctx) != CUDA_SUCCESS || !ctx) return S12_ERR_CUDA;
         g_addr[dev] = p;
+        g_ctx[dev] = ctx;
     }
     *out = g_addr[dev];
     return S12_OK;
@@ -62,24 +85,28 @@ using namespace s12;
 
 extern "C" int s12_gemv_noalloc(const s12_view *v, const uint16_t *x, int B, float *y, uint32_t *err_flag,
                                 void *stream) {
-    if (!v || !x || !y) return S12_ERR_ARG;
+    // the same argument checks and status codes as s12_gemv, first
+    void *out[1] = {y};
+    int rc = gemv_check(v, 1, &x, B, out, nullptr, err_flag);
+    if (rc != S12_OK) return rc;
     if (v->rows > kMaxRows) return S12_ERR_CAPACITY;
     int sms = 0;
     if (device_sms(&sms) != cudaSuccess) return S12_ERR_CUDA;
     if (sms > kMaxSms) return S12_ERR_CAPACITY;
+    const size_t part = gemv_part_bytes(sms);
+    const size_t cnt = gemv_cnt_bytes((v->rows + 15) / 16);
     const size_t need = s12_gemv_ws_bytes(v, B);
-    if (need == 0) return S12_ERR_SHAPE;  // invalid view or batch: s12_gemv reports which
-    if (need > kScratchBytes) return S12_ERR_CAPACITY;
+    if (need != part + cnt || need > kScratchBytes) return S12_ERR_CAPACITY;
     void *ws = nullptr;
-    int rc = scratch_address(&ws);
+    rc = scratch_address(&ws);
     if (rc != S12_OK) return rc;
-    // The arrival counters (the workspace's tail) must start at zero.  A
-    // completed call leaves them zero, but one cut short by an error may not:
-    // clear this call's counters first (an asynchronous memset, no
-    // allocation).  The partial sums need no clearing.
-    const uint64_t cnt = align_up(((v->rows + 15) / 16) * sizeof(uint32_t), kAlign);
-    if (cudaMemsetAsync(static_cast<uint8_t *>(ws) + (need - cnt), 0, cnt,
-                        static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    // The arrival counters (the workspace's tail) must start at zero.  Every
+    // call leaves them zero, a call whose waits gave up included; clearing
+    // this call's counters first (an asynchronous memset, no allocation)
+    // also covers a previous call that never ran to its end.  The partial
+    // sums need no clearing.
+    if (cudaMemsetAsync(static_cast<uint8_t *>(ws) + part, 0, cnt, static_cast<cudaStream_t>(stream)) !=
+        cudaSuccess)
         return S12_ERR_CUDA;
     return s12_gemv(v, x, B, y, ws, need, err_flag, stream);
 }

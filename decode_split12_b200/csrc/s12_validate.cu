@@ -143,26 +143,6 @@ extern "C" int s12_plane_hashes_host(const void *container, size_t bytes, uint64
 namespace s12 {
 namespace {
 
-struct Geometry2 {
-    uint64_t rows, cols, n_tiles, n_esc;
-    uint64_t off_raw, off_code, off_tmeta, off_row_esc, off_esc, total;
-};
-
-Geometry2 geometry2(uint64_t rows, uint64_t cols, uint64_t n_esc) {
-    Geometry2 g;
-    g.rows = rows;
-    g.cols = cols;
-    g.n_tiles = rows * (cols / kTile);
-    g.n_esc = n_esc;
-    g.off_raw = kHeaderBytes;
-    g.off_code = g.off_raw + align_up(rows * cols, kAlign);
-    g.off_tmeta = g.off_code + align_up(rows * cols / 2, kAlign);
-    g.off_row_esc = g.off_tmeta + align_up(2 * g.n_tiles, kAlign);
-    g.off_esc = g.off_row_esc + align_up(4 * (rows + 1), kAlign);
-    g.total = g.off_esc + align_up(2 * n_esc, kAlign);
-    return g;
-}
-
 void wr32(uint8_t *p, uint32_t v) {
     for (int i = 0; i < 4; ++i) p[i] = static_cast<uint8_t>(v >> (8 * i));
 }

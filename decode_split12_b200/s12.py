@@ -36,7 +36,7 @@ S12_FLAG_TIMEOUT = 8
 EXPORTED = (
     "s12_error_string", "s12_device_check", "s12_container_bytes", "s12_encode_ws_bytes", "s12_encode",
     "s12_open", "s12_decode", "s12_gemv_ws_bytes", "s12_gemv", "s12_gemv_multi_ws_bytes", "s12_gemv_multi",
-    "s12_gemv_noalloc", "s12_gemv_swiglu", "s12_gemm_ws_bytes", "s12_gemm_skinny", "s12_gemm_multi_ws_bytes",
+    "s12_gemv_noalloc", "s12_gemv_swiglu", "s12_gemv_bf16", "s12_gemm_ws_bytes", "s12_gemm_skinny", "s12_gemm_multi_ws_bytes",
     "s12_gemm_skinny_multi", "s12_validate_host", "s12_plane_hashes_host", "s12_fnv1a64",
     "s12_to_v2_host", "s12_from_v2_host", "s12_stats_ws_bytes",
     "s12_stats", "s12_bf16_gemv",
@@ -55,6 +55,7 @@ class View(C.Structure):
         ("rows", C.c_uint64), ("cols", C.c_uint64), ("n_tiles", C.c_uint64), ("n_esc", C.c_uint64),
         ("container_bytes", C.c_uint64), ("container", C.c_void_p), ("raw", C.c_void_p),
         ("code", C.c_void_p), ("base", C.c_void_p), ("esc_off", C.c_void_p), ("esc", C.c_void_p),
+        ("version", C.c_uint32), ("reserved", C.c_uint32), ("tmeta", C.c_void_p), ("row_esc", C.c_void_p),
     ]
 
 
@@ -106,6 +107,8 @@ def _lib() -> C.CDLL:
         lib.s12_gemv_noalloc.restype = C.c_int
         lib.s12_gemv_swiglu.argtypes = [C.POINTER(View), _P, C.c_int, _P, _P, _SZ, _P, _P]
         lib.s12_gemv_swiglu.restype = C.c_int
+        lib.s12_gemv_bf16.argtypes = [C.POINTER(View), _P, C.c_int, _P, _P, _SZ, _P, _P]
+        lib.s12_gemv_bf16.restype = C.c_int
         lib.s12_gemv.restype = C.c_int
         lib.s12_gemm_ws_bytes.argtypes = [C.POINTER(View), C.c_int]
         lib.s12_gemm_ws_bytes.restype = _SZ
@@ -257,6 +260,34 @@ def s12_gemv(view: View, x: torch.Tensor, y: torch.Tensor | None = None, ws: tor
     _check(_lib().s12_gemv(C.byref(view), _dptr(x), B, _dptr(y), _dptr(ws), ws.numel(), _dptr(err_flag),
                            _stream(stream)), "s12_gemv")
     return y
+
+
+def s12_gemv_bf16(view: View, x: torch.Tensor, y: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                  err_flag: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """s12_gemv with a BF16 output (round to nearest even), as int16 bits
+    (B x rows)."""
+    x = _u16(x)
+    B = x.shape[0] if x.dim() == 2 else 1
+    if y is None:
+        y = torch.empty((B, view.rows), dtype=torch.int16, device=x.device)
+    if ws is None:
+        ws = gemv_workspace(view, B, x.device)
+    _check(_lib().s12_gemv_bf16(C.byref(view), _dptr(x), B, _dptr(y), _dptr(ws), ws.numel(), _dptr(err_flag),
+                                _stream(stream)), "s12_gemv_bf16")
+    return y
+
+
+def reset_workspace_if_timed_out(err_flag: torch.Tensor | None, *workspaces: torch.Tensor) -> bool:
+    """After a call that was given `err_flag`: if the word shows
+    S12_FLAG_TIMEOUT (a bounded wait inside a kernel gave up), zero the
+    workspaces that call used, so that no stale arrival counter can reach
+    the next call.  Reads the flag back (synchronises).  Returns True if it
+    reset them."""
+    if err_flag is None or not (int(err_flag.item()) & S12_FLAG_TIMEOUT):
+        return False
+    for ws in workspaces:
+        ws.zero_()
+    return True
 
 
 def _view_array(views):

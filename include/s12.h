@@ -92,7 +92,10 @@ extern "C" {
 #define S12_GEMM_MAX_PROBLEMS 16 /* matrices per s12_gemm_skinny_multi call */
 
 /* Host-side description of an opened container.  All pointers are device
- * pointers into the caller's container buffer. */
+ * pointers into the caller's container buffer.  A version 1 container has
+ * `base` and `esc_off` (and NULL tmeta/row_esc); a version 2 container (the
+ * compact tile header of s12_to_v2_host) has `tmeta` and `row_esc` (and NULL
+ * base/esc_off).  Every kernel call reads either version. */
 typedef struct s12_view {
     uint64_t rows;            /* output features (N)                      */
     uint64_t cols;            /* input features (K), multiple of 128      */
@@ -102,9 +105,13 @@ typedef struct s12_view {
     const void *container;    /* start of the container                   */
     const uint8_t *raw;       /* u8 [rows*cols]                           */
     const uint8_t *code;      /* u8 [rows*cols/2]                         */
-    const uint8_t *base;      /* u8 [n_tiles]                             */
-    const uint32_t *esc_off;  /* u32[n_tiles+1]                           */
+    const uint8_t *base;      /* version 1: u8 [n_tiles]                  */
+    const uint32_t *esc_off;  /* version 1: u32[n_tiles+1]                */
     const uint16_t *esc;      /* u16[n_esc]                               */
+    uint32_t version;         /* 1 or 2                                   */
+    uint32_t reserved;        /* 0                                        */
+    const uint16_t *tmeta;    /* version 2: u16[n_tiles], base | count<<8 */
+    const uint32_t *row_esc;  /* version 2: u32[rows+1], escapes before r */
 } s12_view;
 
 typedef struct s12_stats_t {
@@ -160,10 +167,11 @@ int s12_encode(const uint16_t *w, int64_t rows, int64_t cols, void *dst, size_t 
 
 /* Follows: the container layout above, which restates [M] section 1 (the
  * BF16 bit fields) and [T] key points (tile base, escape stream).
- * Validate the 64-byte header of a container (device, `bytes` long) and
- * fill *out with its shape and plane pointers.  Copies the header to the
- * host and so SYNCHRONISES (the legacy default stream).  S12_ERR_CORRUPT on
- * a bad magic, version, tile size, flags, shape or a size above `bytes`. */
+ * Validate the 64-byte header of a container (device, `bytes` long, version
+ * 1 or 2) and fill *out with its shape, version and plane pointers.  Copies
+ * the header to the host and so SYNCHRONISES (the legacy default stream).
+ * S12_ERR_CORRUPT on a bad magic, version, tile size, flags, shape or a size
+ * above `bytes`. */
 int s12_open(const void *container, size_t bytes, s12_view *out);
 
 /* ---- standalone decode ([T] key points: one integer ADD per weight,
@@ -255,6 +263,18 @@ int s12_gemv_multi(const s12_view *views, int count, const uint16_t *const *x, i
  * decode and use the weights at once; the epilogue is this build's own). */
 int s12_gemv_swiglu(const s12_view *v, const uint16_t *x, int B, uint16_t *h, void *ws, size_t ws_bytes,
                     uint32_t *err_flag, void *stream);
+
+/* Follows: [W] "What does 'lossless' mean for LLM weights?" (decode into
+ * registers and multiply at once); the BF16 result is this library's own
+ * option for callers whose next step takes BF16.
+ * s12_gemv with a BF16 output: y[b][n] = bf16_rne(sum_k W[n][k] x[b][k]),
+ * the FP32 sum of s12_gemv rounded to nearest even.
+ *   y:  device BF16, B x rows row-major (2-byte alignment), overwritten.
+ * The rounding adds up to 2^-9 |y| to the error of the FP32 sum (within
+ * 1e-3 sum_k |W[n][k] x[b][k]|), so the result is within that bound plus
+ * 2^-9 |y|.  Other arguments, errors and the workspace as for s12_gemv. */
+int s12_gemv_bf16(const s12_view *v, const uint16_t *x, int B, uint16_t *y, void *ws, size_t ws_bytes,
+                  uint32_t *err_flag, void *stream);
 
 /* The pages have no counterpart of this call: it exists for integration,
  * not for the method.

@@ -125,6 +125,7 @@ def test_argument_checks_need_no_device(lib):
     v.rows, v.cols, v.n_tiles = 4, 128, 4
     for f in ("container", "raw", "code", "base", "esc_off", "esc"):
         setattr(v, f, 0x100000)
+    v.version = 1
     assert lib.s12_gemv(C.byref(v), fake, 0, fake, fake, 1 << 20, None, None) == s12.S12_ERR_SHAPE
     assert lib.s12_gemv(C.byref(v), fake, 9, fake, fake, 1 << 20, None, None) == s12.S12_ERR_SHAPE
     # the GEMV workspace is mandatory and 16-byte aligned
@@ -150,6 +151,7 @@ def test_swiglu_and_gemm_group_argument_checks(lib):
     v.rows, v.cols, v.n_tiles = 24, 128, 24
     for f in ("container", "raw", "code", "base", "esc_off", "esc"):
         setattr(v, f, 0x100000)
+    v.version = 1
     assert lib.s12_gemv_swiglu(C.byref(v), fake, 1, fake, fake, 1 << 20, None, None) == s12.S12_ERR_SHAPE
     v.rows, v.n_tiles = 32, 32
     odd = C.c_void_p(0x100001)

@@ -265,3 +265,91 @@ def test_gemv_inf_activation_at_escape(s12, oracle):
             assert np.isnan(y[0, r])
         else:
             assert y[0, r] == (np.inf if wf[r, col] > 0 else -np.inf), r
+
+
+# ---------------------------------------------------------------------------
+# container version 2 (compact tile header) and the BF16 output
+
+def _v2_blob(oracle, w):
+    """A version 2 container built by the oracle from W, on the device."""
+    from gpu_util import blob_to_dev
+    return blob_to_dev(oracle.encode_v2(w))
+
+
+@pytest.mark.parametrize("checked", [True, False])
+@pytest.mark.parametrize("B", [1, 3, 8])
+@pytest.mark.parametrize("shape", [(1, 128), (3, 384), (149, 640), (300, 1152), (77, 4096), (19, 14336)])
+def test_gemv_v2_small_shapes(s12, oracle, shape, B, checked):
+    """The fused GEMV reading a version 2 container (per tile one u16 of
+    base | escape count, per row one u32 escape offset; [W] English
+    edition, opening summary) matches the FP64 oracle; warps whose range
+    starts in the middle of a row sum the earlier tiles' counts."""
+    r, c = shape
+    w = wl.normal_with_outliers(r, c, 0.02, 0.004, r + 7 * c)
+    x = wl.activations(B, c, B + 1)
+    blob = _v2_blob(oracle, w)
+    view = s12.s12_open(blob)
+    assert view.version == 2
+    flag = new_flag() if checked else None
+    y = s12.s12_gemv(view, to_dev(x), err_flag=flag)
+    torch.cuda.synchronize()
+    yr, sr = oracle.gemv_f64(oracle.encode(w), x)
+    assert_within_tolerance(y.cpu().numpy(), yr, sr)
+    if checked:
+        assert int(flag.item()) == 0
+
+
+def test_gemv_v2_escape_heavy_and_multi(s12, oracle):
+    """Version 2 at 10 % escapes (every tile, some all-escape) in a grouped
+    launch beside a second version 2 matrix; a call that mixes container
+    versions is refused."""
+    w0, _ = wl.escape_stress(0.10, 2, 64, 2048)
+    w1 = wl.student_t_scaled(300, 1152, 3)
+    x0, x1 = wl.activations(4, 2048, 5), wl.activations(4, 1152, 6)
+    b0, b1 = _v2_blob(oracle, w0), _v2_blob(oracle, w1)
+    v0, v1 = s12.s12_open(b0), s12.s12_open(b1)
+    flag = new_flag()
+    ys = s12.s12_gemv_multi([v0, v1], [to_dev(x0), to_dev(x1)], err_flag=flag)
+    torch.cuda.synchronize()
+    for w, x, y in ((w0, x0, ys[0]), (w1, x1, ys[1])):
+        yr, sr = oracle.gemv_f64(oracle.encode(w), x)
+        assert_within_tolerance(y.cpu().numpy(), yr, sr)
+    assert int(flag.item()) == 0
+    v_one = s12.s12_open(s12.s12_encode(to_dev(w1)))
+    with pytest.raises(s12.S12Error):
+        s12.s12_gemv_multi([v0, v_one], [to_dev(x0), to_dev(x1)])
+
+
+@pytest.mark.parametrize("name", ["q", "down"])
+def test_gemv_v2_llama8b_full_size_sampled(s12, oracle, name):
+    """Full-size 8B-layer matrices as version 2 containers (the oracle's own
+    encoding), sampled rows against the FP64 oracle."""
+    mats, xs = wl.llama8b_layer(0, 1, names=[name])
+    w, x = mats[name], xs[name]
+    view = s12.s12_open(_v2_blob(oracle, w))
+    y = s12.s12_gemv(view, to_dev(x))
+    torch.cuda.synchronize()
+    rows = np.unique(np.concatenate([[0, w.shape[0] - 1], wl.rng_for(7, 1).choice(w.shape[0], 46, replace=False)]))
+    yr, sr = oracle.gemv_f64(oracle.encode(w[rows]), x)
+    assert_within_tolerance(y.cpu().numpy()[:, rows], yr, sr)
+
+
+@pytest.mark.parametrize("B", [1, 4, 8])
+@pytest.mark.parametrize("shape", [(3, 384), (300, 1152), (1024, 4096)])
+def test_gemv_bf16_output(s12, oracle, shape, B):
+    """The BF16-output GEMV: each y is the FP32 sum rounded to BF16, so it is
+    within 1e-3 * sum|W x| + 2^-9 |y_ref| of the FP64 oracle (the rounding of
+    a BF16 result adds at most half an ulp, 2^-9 relative)."""
+    r, c = shape
+    w = wl.normal_with_outliers(r, c, 0.02, 0.002, r + c + B)
+    x = wl.activations(B, c, 40 + B)
+    view = s12.s12_open(s12.s12_encode(to_dev(w)))
+    flag = new_flag()
+    yb = s12.s12_gemv_bf16(view, to_dev(x), err_flag=flag)
+    torch.cuda.synchronize()
+    y = wl.bf16_bits_to_f32(yb.cpu().numpy().view(np.uint16)).astype(np.float64)
+    yr, sr = oracle.gemv_f64(oracle.encode(w), x)
+    err = np.abs(y - yr)
+    bound = 1e-3 * sr + 2.0 ** -9 * np.abs(yr)
+    assert (err <= bound).all(), float((err / np.maximum(bound, 1e-300)).max())
+    assert int(flag.item()) == 0

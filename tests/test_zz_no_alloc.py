@@ -86,6 +86,7 @@ def test_noalloc_rejects_oversized(s12):
     v.rows, v.cols, v.n_tiles = (1 << 20) + 16, 128, (1 << 20) + 16
     for f in ("container", "raw", "code", "base", "esc_off", "esc"):
         setattr(v, f, 0x100000)
+    v.version = 1
     x = torch.zeros((1, 128), dtype=torch.int16, device="cuda")
     y = torch.zeros((1, 16), dtype=torch.float32, device="cuda")
     rc = s12.lib().s12_gemv_noalloc(C.byref(v), C.c_void_p(x.data_ptr()), 1, C.c_void_p(y.data_ptr()), None, None)
