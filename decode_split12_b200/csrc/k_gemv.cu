@@ -88,8 +88,8 @@ constexpr int kOutF32 = kGemvOutF32, kOutSwiglu = kGemvOutSwiglu, kOutBf16 = kGe
 
 // One matrix of a grouped call.
 struct __align__(64) Problem {
-    CUtensorMap tm_raw;   // u8 {128, R, T} (strides K, 128), box {128, 16, 2}, 128-byte swizzle
-    CUtensorMap tm_code;  // u8 {64, R, T} (strides K/2, 64), box {64, 16, 2}
+    CUtensorMap tm_raw;   // u8 {128, T, R} (strides 128, K), box {128, 2, 16}, 128-byte swizzle
+    CUtensorMap tm_code;  // u8 {64, T, R} (strides 64, K/2), box {64, 2, 16}, 64-byte swizzle
     const void *meta;     // version 1: base u8[n_tiles]; version 2: (base | count << 8) u16[n_tiles]
     const uint32_t *off;  // version 1: esc_off u32[n_tiles + 1]; version 2: row_esc u32[R + 1]
     const uint16_t *esc;
@@ -111,6 +111,12 @@ struct __align__(64) Params {
     int n_problems, B;
     int n_units;    // warps in the grid
 };
+
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+    return v;
+}
 
 __device__ __forceinline__ uint4 lds128(uint32_t a) {
     uint4 v;
@@ -203,35 +209,54 @@ __device__ __forceinline__ void issue(const Params &pr, const Cur &c, uint32_t s
     const Problem &m = pr.prob[c.p];
     const uint64_t pol = policy_evict_first();
     mbar_expect_tx_s(bar, kStageBytes);
-    tma3d(st, &m.tm_raw, 0, c.grp * kRowsPerGroup, c.j, bar, pol);
-    tma3d(st + kRawStage, &m.tm_code, 0, c.grp * kRowsPerGroup, c.j, bar, pol);
+    tma3d(st, &m.tm_raw, 0, c.j, c.grp * kRowsPerGroup, bar, pol);
+    tma3d(st + kRawStage, &m.tm_code, 0, c.j, c.grp * kRowsPerGroup, bar, pol);
 }
 
 // ---------------------------------------------------------------------------
-// Metadata.  Per stage the lane loads one word for each of its rows (row r of
-// matrix m, tiles j .. j+len-1); the quad's four words are, by lane q:
-//   version 1:  base[t], base[t+1], esc_off[t+1], esc_off[t+2]   (t = r*T + j)
-//   version 2:  tmeta[t], tmeta[t+1], -, -
-// Rows past the end read as 0 (no escapes).
+// Metadata.  Lane (g, q) of a stage works on tile tq = q / 2 of the stage
+// (its columns 64 (q % 2) .. +63 of that tile) for rows g and g+8, so it needs
+// per row one base and the tile row's escape span [s, e).  They are loaded a
+// stage ahead into a Meta (rows past the end and lanes past the stage's last
+// tile read as base 0 with an empty span):
+//   version 1:  base[t], esc_off[t], esc_off[t+1]     (t = r*T + j + tq)
+//   version 2:  tmeta of the stage's two tiles, and the row's escape offset
+//               row_esc[r] when the stage starts a row group; the spans
+//               follow from a running offset per row.
+struct Meta {
+    uint32_t a0, a1, a2;  // row g
+    uint32_t b0, b1, b2;  // row g + 8
+};
+
+// (the loaded words are kept as they are: any arithmetic on them here would
+// make the warp wait for the loads a stage early)
 template <int V>
-__device__ __forceinline__ uint32_t load_item(const Problem &m, int r, int j, int len, int q) {
-    if (r >= m.R) return 0;
+__device__ __forceinline__ void load_row_meta(const Problem &m, int r, int j, int len, int tq, bool seg_start,
+                                              uint32_t &w0, uint32_t &w1, uint32_t &w2) {
+    w0 = w1 = w2 = 0u;
+    if (r >= m.R) return;
     const size_t t0 = static_cast<size_t>(r) * m.T + j;
     if (V == 1) {
-        if (q < 2) return q < len ? static_cast<uint32_t>(__ldg(static_cast<const uint8_t *>(m.meta) + t0 + q)) : 0u;
-        return q - 2 < len ? __ldg(m.off + t0 + 1 + (q - 2)) : 0u;
+        if (tq < len) {
+            w0 = __ldg(static_cast<const uint8_t *>(m.meta) + t0 + tq);
+            w1 = __ldg(m.off + t0 + tq);
+            w2 = __ldg(m.off + t0 + tq + 1);
+        }
+    } else {
+        const uint16_t *tm = static_cast<const uint16_t *>(m.meta) + t0;
+        w0 = __ldg(tm);
+        if (len > 1) w1 = __ldg(tm + 1);
+        if (seg_start) w2 = __ldg(m.off + r);
     }
-    return q < len ? static_cast<uint32_t>(__ldg(static_cast<const uint16_t *>(m.meta) + t0 + q)) : 0u;
 }
 
-// Escapes before tile (r, j) in the stream, for a segment that starts at
-// tile j (version 2: only the row start; the caller adds the earlier tiles'
-// counts when j > 0).
 template <int V>
-__device__ __forceinline__ uint32_t load_start(const Problem &m, int r, int j) {
-    if (r >= m.R) return 0;
-    if (V == 1) return __ldg(m.off + static_cast<size_t>(r) * m.T + j);
-    return __ldg(m.off + r);
+__device__ __forceinline__ Meta load_meta(const Problem &m, const Cur &c, int len, int g, int tq, bool seg_start) {
+    const int rA = c.grp * kRowsPerGroup + g;
+    Meta r;
+    load_row_meta<V>(m, rA, c.j, len, tq, seg_start, r.a0, r.a1, r.a2);
+    load_row_meta<V>(m, rA + 8, c.j, len, tq, seg_start, r.b0, r.b1, r.b2);
+    return r;
 }
 
 // Escape counts of tiles 0 .. j-1 of row r (version 2), summed across the
@@ -247,81 +272,47 @@ __device__ __forceinline__ uint32_t prefix_count_v2(const Problem &m, int r, int
     return s;
 }
 
-struct Meta {
-    uint32_t a, b;    // the lane's words for rows g and g+8
-    uint32_t sa, sb;  // escapes before the stage's first tile (segment starts only)
-};
-
+// A row's base and escape span [s, e) for the lane's tile; `run` is the
+// row's escape offset at the stage's first tile (version 2), advanced past
+// the stage.
 template <int V>
-__device__ __forceinline__ Meta load_meta(const Problem &m, const Cur &c, int len, int g, int q, bool seg_start) {
-    const int rA = c.grp * kRowsPerGroup + g, rB = rA + 8;
-    Meta r;
-    r.a = load_item<V>(m, rA, c.j, len, q);
-    r.b = load_item<V>(m, rB, c.j, len, q);
-    r.sa = seg_start ? load_start<V>(m, rA, c.j) : 0u;
-    r.sb = seg_start ? load_start<V>(m, rB, c.j) : 0u;
-    return r;
-}
-
-// Base and escape-span end of tile t of the stage for one row, from the
-// quad's words (w = the lane's word for that row, off = the running offset).
-template <int V>
-__device__ __forceinline__ void tile_meta(uint32_t w, int qb, int t, uint32_t off, uint32_t &base, uint32_t &end) {
-    const uint32_t v = __shfl_sync(0xFFFFFFFFu, w, qb + t);
-    base = v & 0xFFu;
-    if (V == 1)
-        end = __shfl_sync(0xFFFFFFFFu, w, qb + 2 + t);
-    else
-        end = off + (v >> 8);
+__device__ __forceinline__ void row_span(uint32_t w0, uint32_t w1, uint32_t w2, int tq, uint32_t &run, uint32_t &base,
+                                         uint32_t &s, uint32_t &e) {
+    if (V == 1) {
+        base = w0;
+        s = w1;
+        e = w2;
+    } else {
+        const uint32_t c0 = w0 >> 8, c1 = w1 >> 8;
+        base = (tq ? w1 : w0) & 0xFFu;
+        s = run + (tq ? c0 : 0u);
+        e = s + (tq ? c1 : c0);
+        run += c0 + c1;
+    }
 }
 
 // ---------------------------------------------------------------------------
 // Escapes.
 
-__device__ __forceinline__ uint2 esc_mask(uint32_t a, uint32_t b) {
-    return make_uint2(escape_nibbles(a), escape_nibbles(b));
+// Escape-nibble counts of the lane's four 16-weight chunks of one row, one
+// byte each (code words cw[0..3]: chunk c is cw[c/2].{x,y} or .{z,w}).
+__device__ __forceinline__ uint32_t chunk_counts(uint4 c01, uint4 c23) {
+    return __popc(escape_nibbles(c01.x) | (escape_nibbles(c01.y) >> 1)) |
+           (__popc(escape_nibbles(c01.z) | (escape_nibbles(c01.w) >> 1)) << 8) |
+           (__popc(escape_nibbles(c23.x) | (escape_nibbles(c23.y) >> 1)) << 16) |
+           (__popc(escape_nibbles(c23.z) | (escape_nibbles(c23.w) >> 1)) << 24);
 }
 
-// Escapes of one tile row for this lane: the masks of its two halves, the
-// stream index of its first escape in each, and the end of the row's span.
-// Called by all 32 lanes; the four lanes of a quad share the row and rank
-// their escapes in chunk order (lane q = 0..3, half 0 then half 1).  The
-// tile's code-15 count is checked against its span.
-struct EscRow {
-    uint2 m0, m1;
-    uint32_t s0, s1, limit;
-};
-
-__device__ __forceinline__ EscRow prepare_row(uint4 c, uint32_t lo, uint32_t hi, uint32_t n_esc, uint32_t *err,
-                                              int q) {
-    EscRow e;
-    e.m0 = esc_mask(c.x, c.y);
-    e.m1 = esc_mask(c.z, c.w);
-    const uint32_t n0 = __popc(e.m0.x) + __popc(e.m0.y);
-    const uint32_t n = n0 + __popc(e.m1.x) + __popc(e.m1.y);
-    uint32_t incl = n;
-#pragma unroll
-    for (int d = 1; d < 4; d <<= 1) {
-        const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, d, 4);
-        if (q >= d) incl += v;
-    }
-    const uint32_t tot = __shfl_sync(0xFFFFFFFFu, incl, 3, 4);
-    e.s0 = lo + incl - n;
-    e.s1 = e.s0 + n0;
-    e.limit = lo <= hi ? min(hi, n_esc) : 0u;
-    if (q == 0 && tot != hi - lo) raise_flag(err, S12_FLAG_ESC_COUNT);
-    return e;
-}
-
-// A half with escapes: put the exact value of each escaped weight in place,
-// reading the stream from index `idx`; reads at or past `limit` are skipped
-// and flagged.  The decoded words go through the lane's 32-byte shared
-// scratch `sc`, so a weight is replaced by one 16-bit store at its position.
-// With base <= 240, base + 15 stays inside its byte and the other weights of
-// the half are already right; a base of 241 could carry into the next byte,
-// so such halves are decoded again with the escape nibbles cleared first.
-__device__ __forceinline__ void fix_half(uint32_t (&w)[8], uint4 raw, uint2 code, uint2 m, uint32_t base, uint32_t idx,
-                                      uint32_t limit, const uint16_t *__restrict__ esc, uint32_t *err, uint32_t sc) {
+// A chunk with escapes: put the exact value of each escaped weight in place,
+// taking stream index `idx` on; reads at or past `limit` are skipped and
+// flagged.  The decoded words go through the lane's 32-byte shared scratch
+// `sc`, so a weight is replaced by one 16-bit store at its position.  With
+// base <= 240, base + 15 stays inside its byte and the other weights of the
+// chunk are already right; a base of 241 could carry into the next byte, so
+// such chunks are decoded again with the escape nibbles cleared first.
+__device__ __forceinline__ void fix_chunk(uint32_t (&w)[8], uint4 raw, uint2 code, uint2 m, uint32_t base,
+                                          uint32_t idx, uint32_t limit, const uint16_t *__restrict__ esc,
+                                          uint32_t *err, uint32_t sc) {
     if (base > static_cast<uint32_t>(kMaxBase - 1))
         decode16(raw, make_uint2(clear_escapes(code.x, m.x), clear_escapes(code.y, m.y)), base * 0x01010101u, w);
     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sc), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
@@ -329,7 +320,7 @@ __device__ __forceinline__ void fix_half(uint32_t (&w)[8], uint4 raw, uint2 code
     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sc + 16), "r"(w[4]), "r"(w[5]), "r"(w[6]),
                  "r"(w[7])
                  : "memory");
-    // nibble j of the half is 15  <=>  bit 4j+3 of the 64-bit mask
+    // nibble j of the chunk is 15  <=>  bit 4j+3 of the 64-bit mask
     uint64_t mm = (static_cast<uint64_t>(m.y) << 32) | m.x;
     while (mm) {
         const int j = (__ffsll(static_cast<long long>(mm)) - 1) >> 2;
@@ -355,16 +346,16 @@ __device__ __forceinline__ void fix_half(uint32_t (&w)[8], uint4 raw, uint2 code
 // ---------------------------------------------------------------------------
 // Products.
 
-// The lane's 16 activations of half h (batch row of xl, columns 32q + 16h ..
-// of the tile at xl), read through the L1 cache.
-__device__ __forceinline__ void load_x(uint32_t (&xw)[8], const uint16_t *xl, int h) {
-    const uint4 *src = reinterpret_cast<const uint4 *>(xl + h * 16);
+// The lane's 16 activations of chunk c (batch row and first column at xl),
+// read through the L1 cache.
+__device__ __forceinline__ void load_x(uint32_t (&xw)[8], const uint16_t *xl, int c) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(xl + c * 16);
     const uint4 a = __ldg(src), b = __ldg(src + 1);
     xw[0] = a.x; xw[1] = a.y; xw[2] = a.z; xw[3] = a.w;
     xw[4] = b.x; xw[5] = b.y; xw[6] = b.z; xw[7] = b.w;
 }
 
-// One half of a block: four m16n8k16 products of rows g / g+8 with x.
+// One chunk: four m16n8k16 products of rows g / g+8 with x.
 __device__ __forceinline__ void half_mma(float (&acc)[4], const uint32_t (&wa)[8], const uint32_t (&wb)[8],
                                          const uint32_t (&xw)[8]) {
 #pragma unroll
@@ -474,7 +465,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
     extern __shared__ uint8_t smem_raw[];
     const uint32_t sb = (smem_addr(smem_raw) + 1023u) & ~1023u;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = lane >> 2, q = lane & 3, qb = lane & ~3;
+    const int g = lane >> 2, q = lane & 3, tq = q >> 1, qh = q & 1;
     const uint32_t bars = sb + static_cast<uint32_t>(warp) * kStages * 8u;
     const uint32_t ring = sb + kRingOff + static_cast<uint32_t>(warp) * kStages * kStageBytes;
     if (threadIdx.x == 0) grid_launch_dependents();
@@ -507,32 +498,44 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
     }
 
     int lenc = stage_len(pr, cc);
-    Meta mc = load_meta<V>(pr.prob[cc.p], cc, lenc, g, q, true);
-    if (V == 2 && cc.j > 0) {
-        mc.sa += prefix_count_v2(pr.prob[cc.p], cc.grp * kRowsPerGroup + g, cc.j, q);
-        mc.sb += prefix_count_v2(pr.prob[cc.p], cc.grp * kRowsPerGroup + g + 8, cc.j, q);
+    Meta mc = load_meta<V>(pr.prob[cc.p], cc, lenc, g, tq, true);
+    uint32_t runA = 0, runB = 0;  // version 2: the rows' escape offsets at the current stage
+    if (V == 2) {
+        runA = mc.a2;
+        runB = mc.b2;
+        if (cc.j > 0) {
+            runA += prefix_count_v2(pr.prob[cc.p], cc.grp * kRowsPerGroup + g, cc.j, q);
+            runB += prefix_count_v2(pr.prob[cc.p], cc.grp * kRowsPerGroup + g + 8, cc.j, q);
+        }
     }
     Cur cn = cc;  // the stage after it
     advance(cn, lenc, pr);
+
     int gp = cc.p, ggrp = cc.grp;  // the row group being accumulated
-    uint32_t offA = mc.sa, offB = mc.sb;
     const int G0 = group_id(pr, gp, ggrp);
     grid_dependency_wait();  // x, y and the workspace may belong to earlier kernels
     const int gx = g < pr.B ? g : 0;  // batch rows past B repeat row 0; their outputs are dropped
-    // the lane's shared-memory offsets inside a tile (raw rows are 128-byte swizzled)
-    const uint32_t oA0 = g * 128 + (((2 * q) ^ g) << 4), oA1 = g * 128 + (((2 * q + 1) ^ g) << 4);
-    const uint32_t oCA = kRawStage + g * 64 + 16 * q;
+    // The lane's shared-memory places (stage layout [row][tile][bytes]): raw
+    // row g of its tile at oR (row g+8 2048 bytes on), 16-byte chunk k of it
+    // at ((k ^ rsw) << 4); code row g at oC (row g+8 1024 bytes on), 16-byte
+    // piece k at ((k ^ csw) << 4).  With the copy engine's 128-byte (raw) and
+    // 64-byte (code) swizzles, every 16-byte read of a quarter warp hits its
+    // own banks.
+    const uint32_t oR = static_cast<uint32_t>(2 * g + tq) * 128u, rsw = static_cast<uint32_t>(2 * g + tq) & 7u;
+    const uint32_t oC = kRawStage + static_cast<uint32_t>(2 * g + tq) * 64u, csw = static_cast<uint32_t>(g) & 3u;
+    const uint32_t oC0 = oC + ((static_cast<uint32_t>(2 * qh) ^ csw) << 4);
+    const uint32_t oC1 = oC + ((static_cast<uint32_t>(2 * qh + 1) ^ csw) << 4);
 
-    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};  // one chain per half
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};  // two chains
     int consumed = 0;  // stages consumed so far
     bool ok = true;
     while (cc.left > 0) {
         // metadata of the next stage, one stage ahead
         int lenn = 0;
-        Meta mn = {0u, 0u, 0u, 0u};
+        Meta mn = {0u, 0u, 0u, 0u, 0u, 0u};
         if (cn.left > 0) {
             lenn = stage_len(pr, cn);
-            mn = load_meta<V>(pr.prob[cn.p], cn, lenn, g, q, cn.j == 0);
+            mn = load_meta<V>(pr.prob[cn.p], cn, lenn, g, tq, cn.j == 0);
         }
         if (cc.p != gp || cc.grp != ggrp) {
             finish_group(pr, sum_halves(acc), gp, ggrp, G0);
@@ -540,8 +543,10 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
             for (int k = 0; k < 4; ++k) acc[0][k] = acc[1][k] = 0.f;
             gp = cc.p;
             ggrp = cc.grp;
-            offA = mc.sa;
-            offB = mc.sb;
+            if (V == 2) {
+                runA = mc.a2;
+                runB = mc.b2;
+            }
         }
         const int s = consumed & 1;
         const uint32_t bar = bars + 8u * s;
@@ -552,74 +557,113 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
         }
         const Problem &m = pr.prob[cc.p];
         const uint32_t st = ring + s * kStageBytes;
-        const uint16_t *xrow = m.x + static_cast<size_t>(gx) * m.K + 32 * q + static_cast<size_t>(cc.j) * kTile;
+        const bool live = tq < lenc;  // the lane's tile belongs to this stage
+        uint32_t bA, sA, eA, bB, sB, eB;
+        row_span<V>(mc.a0, mc.a1, mc.a2, tq, runA, bA, sA, eA);
+        row_span<V>(mc.b0, mc.b1, mc.b2, tq, runB, bB, sB, eB);
+
+        uint4 cA0 = make_uint4(0, 0, 0, 0), cA1 = cA0, cB0 = cA0, cB1 = cA0;
+        if (live) {
+            cA0 = lds128(st + oC0);
+            cA1 = lds128(st + oC1);
+            cB0 = lds128(st + oC0 + 1024);
+            cB1 = lds128(st + oC1 + 1024);
+        }
+        bool esc = (eA != sA) || (eB != sB);
+        if (CHECK) {
+            // every tile row's code-15 count against its span (the two lanes
+            // of a pair hold the row's two halves)
+            const uint32_t ccA = chunk_counts(cA0, cA1), ccB = chunk_counts(cB0, cB1);
+            const uint32_t totA = (ccA * 0x01010101u) >> 24, totB = (ccB * 0x01010101u) >> 24;
+            const uint32_t pairA = __shfl_xor_sync(0xFFFFFFFFu, totA, 1), pairB = __shfl_xor_sync(0xFFFFFFFFu, totB, 1);
+            if (live && qh == 0 && (totA + pairA != eA - sA || totB + pairB != eB - sB))
+                raise_flag(pr.err, S12_FLAG_ESC_COUNT);
+            esc = esc || (ccA | ccB) != 0;
+            if (bA > static_cast<uint32_t>(kMaxBase) || bB > static_cast<uint32_t>(kMaxBase))
+                raise_flag(pr.err, S12_FLAG_BASE);
+        }
+        const bool anyesc = __any_sync(0xFFFFFFFFu, esc);
+        const uint32_t B4A = bA * 0x01010101u, B4B = bB * 0x01010101u;
+        const uint16_t *xl = m.x + static_cast<size_t>(gx) * m.K + static_cast<size_t>(cc.j + tq) * kTile + 64 * qh;
+        const uint32_t oRA = st + oR, oRB = oRA + 2048;
+        if (!anyesc) {
+            // no escapes in the stage: straight decode and products, the
+            // loop unrolled (this is the hot code)
 #pragma unroll
-        for (int t = 0; t < kNT; ++t) {
-            if (t >= lenc) break;
-            const uint32_t tt = st + t * kRawTile, tc = st + t * kCodeTile;
-            const uint4 rA0 = lds128(tt + oA0), rA1 = lds128(tt + oA1);
-            const uint4 rB0 = lds128(tt + oA0 + 8 * 128), rB1 = lds128(tt + oA1 + 8 * 128);
-            const uint4 cA = lds128(tc + oCA), cB = lds128(tc + oCA + 8 * 64);
-            if (t == lenc - 1) {
-                // the stage is in registers: hand it back to the copy engine
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                __syncwarp();
-                if (pc.left > 0) {
-                    const int len = stage_len(pr, pc);
-                    if (lane == 0) issue(pr, pc, st, bar);
-                    advance(pc, len, pr);
-                    ++issued;
+            for (int c = 0; c < 4; ++c) {
+                uint4 rA = make_uint4(0, 0, 0, 0), rB = rA;
+                if (live) {
+                    rA = lds128(oRA + ((static_cast<uint32_t>(4 * qh + c) ^ rsw) << 4));
+                    rB = lds128(oRB + ((static_cast<uint32_t>(4 * qh + c) ^ rsw) << 4));
                 }
+                if (c == 3) {
+                    // the stage is in registers: hand it back to the copy engine
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    if (pc.left > 0) {
+                        const int len = stage_len(pr, pc);
+                        if (lane == 0) issue(pr, pc, st, bar);
+                        advance(pc, len, pr);
+                        ++issued;
+                    }
+                }
+                uint32_t xw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+                if (live) load_x(xw, xl, c);
+                const uint4 kA4 = c < 2 ? cA0 : cA1, kB4 = c < 2 ? cB0 : cB1;
+                const uint2 kA = (c & 1) ? make_uint2(kA4.z, kA4.w) : make_uint2(kA4.x, kA4.y);
+                const uint2 kB = (c & 1) ? make_uint2(kB4.z, kB4.w) : make_uint2(kB4.x, kB4.y);
+                uint32_t wa[8], wb[8];
+                decode16(rA, kA, B4A, wa);
+                decode16(rB, kB, B4B, wb);
+                half_mma(acc[c & 1], wa, wb, xw);
             }
-            uint32_t bA, eA, bB, eB;
-            tile_meta<V>(mc.a, qb, t, offA, bA, eA);
-            tile_meta<V>(mc.b, qb, t, offB, bB, eB);
-            bool esc = (eA != offA) || (eB != offB);
-            if (CHECK) {
-                esc = esc || (escape_nibbles(cA.x) | escape_nibbles(cA.y) | escape_nibbles(cA.z) | escape_nibbles(cA.w) |
-                              escape_nibbles(cB.x) | escape_nibbles(cB.y) | escape_nibbles(cB.z) |
-                              escape_nibbles(cB.w)) != 0;
-                if (bA > static_cast<uint32_t>(kMaxBase) || bB > static_cast<uint32_t>(kMaxBase))
-                    raise_flag(pr.err, S12_FLAG_BASE);
+        } else {
+            // some tile row of the stage has escapes: one compact loop over
+            // the chunks (rare code, kept small), the stage held until its end
+            const uint32_t ccA = chunk_counts(cA0, cA1), ccB = chunk_counts(cB0, cB1);
+            // the lane's first escape in each row: the first half of a tile
+            // row counts from the span's start, the second half back from its
+            // end (its escapes are the row's last ones)
+            uint32_t iA = qh ? eA - ((ccA * 0x01010101u) >> 24) : sA;
+            uint32_t iB = qh ? eB - ((ccB * 0x01010101u) >> 24) : sB;
+            const uint32_t limA = sA <= eA ? min(eA, m.n_esc) : 0u, limB = sB <= eB ? min(eB, m.n_esc) : 0u;
+            const uint32_t scr = sb + kRingOff + kWarps * kStages * kStageBytes + threadIdx.x * 32u;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint4 rA = make_uint4(0, 0, 0, 0), rB = rA;
+                uint2 kA = make_uint2(0, 0), kB = kA;
+                uint32_t xw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+                if (live) {
+                    rA = lds128(oRA + ((static_cast<uint32_t>(4 * qh + c) ^ rsw) << 4));
+                    rB = lds128(oRB + ((static_cast<uint32_t>(4 * qh + c) ^ rsw) << 4));
+                    // chunk c's 8 code bytes: 16-byte piece c / 2 (swizzled), half c % 2
+                    const uint32_t piece = st + oC + ((static_cast<uint32_t>(2 * qh + (c >> 1)) ^ csw) << 4) + 8u * (c & 1);
+                    kA = lds64(piece);
+                    kB = lds64(piece + 1024);
+                    load_x(xw, xl, c);
+                }
+                uint32_t wa[8], wb[8];
+                decode16(rA, kA, B4A, wa);
+                decode16(rB, kB, B4B, wb);
+                const uint2 mA = make_uint2(escape_nibbles(kA.x), escape_nibbles(kA.y));
+                const uint2 mB = make_uint2(escape_nibbles(kB.x), escape_nibbles(kB.y));
+                if (mA.x | mA.y) fix_chunk(wa, rA, kA, mA, bA, iA, limA, m.esc, pr.err, scr);
+                if (mB.x | mB.y) fix_chunk(wb, rB, kB, mB, bB, iB, limB, m.esc, pr.err, scr);
+                iA += (ccA >> (8 * c)) & 0xFFu;
+                iB += (ccB >> (8 * c)) & 0xFFu;
+                if (c & 1)
+                    half_mma(acc[1], wa, wb, xw);
+                else
+                    half_mma(acc[0], wa, wb, xw);
             }
-            const uint16_t *xl = xrow + t * kTile;
-            const uint32_t B4A = bA * 0x01010101u, B4B = bB * 0x01010101u;
-            uint32_t xw[8], wa[8], wb[8];
-            if (!__any_sync(0xFFFFFFFFu, esc)) {
-                // no escapes in the block: straight decode and products
-                load_x(xw, xl, 0);
-                decode16(rA0, make_uint2(cA.x, cA.y), B4A, wa);
-                decode16(rB0, make_uint2(cB.x, cB.y), B4B, wb);
-                half_mma(acc[0], wa, wb, xw);
-                load_x(xw, xl, 1);
-                decode16(rA1, make_uint2(cA.z, cA.w), B4A, wa);
-                decode16(rB1, make_uint2(cB.z, cB.w), B4B, wb);
-                half_mma(acc[1], wa, wb, xw);
-            } else {
-                // some row of the block has escapes: rank them per row (quad
-                // shuffles), decode, patch the escaped weights, multiply
-                const uint32_t scr = sb + kRingOff + kWarps * kStages * kStageBytes + threadIdx.x * 32u;
-                const EscRow xa = prepare_row(cA, offA, eA, m.n_esc, pr.err, q);
-                const EscRow xb = prepare_row(cB, offB, eB, m.n_esc, pr.err, q);
-                load_x(xw, xl, 0);
-                decode16(rA0, make_uint2(cA.x, cA.y), B4A, wa);
-                decode16(rB0, make_uint2(cB.x, cB.y), B4B, wb);
-                if (xa.m0.x | xa.m0.y)
-                    fix_half(wa, rA0, make_uint2(cA.x, cA.y), xa.m0, bA, xa.s0, xa.limit, m.esc, pr.err, scr);
-                if (xb.m0.x | xb.m0.y)
-                    fix_half(wb, rB0, make_uint2(cB.x, cB.y), xb.m0, bB, xb.s0, xb.limit, m.esc, pr.err, scr);
-                half_mma(acc[0], wa, wb, xw);
-                load_x(xw, xl, 1);
-                decode16(rA1, make_uint2(cA.z, cA.w), B4A, wa);
-                decode16(rB1, make_uint2(cB.z, cB.w), B4B, wb);
-                if (xa.m1.x | xa.m1.y)
-                    fix_half(wa, rA1, make_uint2(cA.z, cA.w), xa.m1, bA, xa.s1, xa.limit, m.esc, pr.err, scr);
-                if (xb.m1.x | xb.m1.y)
-                    fix_half(wb, rB1, make_uint2(cB.z, cB.w), xb.m1, bB, xb.s1, xb.limit, m.esc, pr.err, scr);
-                half_mma(acc[1], wa, wb, xw);
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (pc.left > 0) {
+                const int len = stage_len(pr, pc);
+                if (lane == 0) issue(pr, pc, st, bar);
+                advance(pc, len, pr);
+                ++issued;
             }
-            offA = eA;
-            offB = eB;
         }
         ++consumed;
         cc = cn;
@@ -636,7 +680,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
     // group's counter returns to zero, then let the copies still in flight
     // land before the warp exits.
     const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int left = cc.left + (cc.j > 0 ? cc.j : 0);;) {
+    for (int left = cc.left + cc.j;;) {
         finish_group(pr, z, gp, ggrp, G0);
         // blocks of this warp's range after the group just finished
         left -= pr.prob[gp].T;
@@ -693,10 +737,10 @@ int run(const s12_view *views, int count, const uint16_t *const *x, int B, void 
         const s12_view *v = views + i;
         gemv::Problem &m = pr.prob[i];
         const uint64_t R = v->rows, K = v->cols, T = K / kTile;
-        if (make_tmap_u8_3d(&m.tm_raw, v->raw, 128, R, T, K, 128, 128, gemv::kRowsPerGroup, gemv::kNT, 128) !=
+        if (make_tmap_u8_3d(&m.tm_raw, v->raw, 128, T, R, 128, K, 128, gemv::kNT, gemv::kRowsPerGroup, 128) !=
             S12_OK)
             return S12_ERR_CUDA;
-        if (make_tmap_u8_3d(&m.tm_code, v->code, 64, R, T, K / 2, 64, 64, gemv::kRowsPerGroup, gemv::kNT, 0) !=
+        if (make_tmap_u8_3d(&m.tm_code, v->code, 64, T, R, 64, K / 2, 64, gemv::kNT, gemv::kRowsPerGroup, 64) !=
             S12_OK)
             return S12_ERR_CUDA;
         m.meta = V == 1 ? static_cast<const void *>(v->base) : static_cast<const void *>(v->tmeta);
