@@ -1,66 +1,9 @@
-// k_misc.cu -- exponent-histogram kernel for s12_stats and the plain BF16
-// GEMV used as the uncompressed comparison point.
+// k_misc.cu -- the plain BF16 GEMV used as the uncompressed comparison point
+// (the exponent histogram of s12_stats runs on the decode kernel, k_decode.cu).
 #include "s12_device.cuh"
 #include "s12_launch.h"
 
 namespace s12 {
-
-// ---------------------------------------------------------------------------
-// Exponent histogram of the decoded weights ("你的 bf16 模型,有 5 個 bit 是廢的",
-// section 1: the exponent field carries about 2.6 of its 8 bits).  Decodes
-// 16 weights per lane exactly as s12_decode does and counts their exponent
-// fields in a per-CTA shared histogram.
-__global__ void __launch_bounds__(256) exp_hist_kernel(s12_view v, unsigned long long *hist) {
-    __shared__ uint32_t s_hist[256];
-    s_hist[threadIdx.x] = 0;
-    __syncthreads();
-    const int lane = threadIdx.x & 31;
-    const uint64_t n16 = v.rows * v.cols / 16;
-    const uint64_t warp = (static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-    const uint64_t n_warps = (static_cast<uint64_t>(gridDim.x) * blockDim.x) >> 5;
-    for (uint64_t wc = warp; wc < (n16 + 31) / 32; wc += n_warps) {
-        const uint64_t q = wc * 32 + lane;
-        const bool active = q < n16;
-        uint4 raw = make_uint4(0, 0, 0, 0);
-        uint2 code = make_uint2(0, 0);
-        uint32_t b = 0, lo = 0, hi = 0;
-        if (active) {
-            raw = __ldg(reinterpret_cast<const uint4 *>(v.raw) + q);
-            code = __ldg(reinterpret_cast<const uint2 *>(v.code) + q);
-            b = __ldg(v.base + (q >> 3));
-            lo = __ldg(v.esc_off + (q >> 3));
-            hi = __ldg(v.esc_off + (q >> 3) + 1);
-        }
-        const uint32_t B4 = b * 0x01010101u;
-        const uint32_t m0 = escape_nibbles(code.x), m1 = escape_nibbles(code.y);
-        uint32_t w[8];
-        decode16(raw, code, B4, w);
-        if (__ballot_sync(0xFFFFFFFFu, (m0 | m1) != 0))
-            fix_escapes(w, raw, code, B4, m0, m1, lo, hi, active, v.n_esc, v.esc, nullptr);
-        if (active) {
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                atomicAdd(&s_hist[(w[k] >> 7) & 0xFFu], 1u);
-                atomicAdd(&s_hist[(w[k] >> 23) & 0xFFu], 1u);
-            }
-        }
-    }
-    __syncthreads();
-    if (s_hist[threadIdx.x]) atomicAdd(hist + threadIdx.x, static_cast<unsigned long long>(s_hist[threadIdx.x]));
-}
-
-int launch_stats_hist(const s12_view *v, unsigned long long *hist, cudaStream_t stream) {
-    if (v->version != 1) return S12_ERR_ARG;
-    int sms = 0;
-    if (device_sms(&sms) != cudaSuccess) return S12_ERR_CUDA;
-    if (cudaMemsetAsync(hist, 0, 256 * sizeof(unsigned long long), stream) != cudaSuccess) return S12_ERR_CUDA;
-    const uint64_t need = (v->rows * v->cols / 16 + 255) / 256;
-    uint64_t grid = static_cast<uint64_t>(sms) * 4;
-    if (grid > need) grid = need;
-    if (grid == 0) grid = 1;
-    exp_hist_kernel<<<static_cast<unsigned>(grid), 256, 0, stream>>>(*v, hist);
-    return cudaGetLastError() == cudaSuccess ? S12_OK : S12_ERR_CUDA;
-}
 
 // ---------------------------------------------------------------------------
 // Plain BF16 GEMV (uncompressed baseline).  One warp per row, 128-bit loads

@@ -399,7 +399,7 @@ int s12_stats(const s12_view *v, s12_stats_t *out, void *ws, size_t ws_bytes, vo
     out->n_esc = v->n_esc;
     out->container_bytes = v->container_bytes;
     out->payload_bytes = nw + nw / 2;
-    out->header_bytes = v->n_tiles * 5;
+    out->header_bytes = v->version == 1 ? v->n_tiles * 5 : v->n_tiles * 2 + 4 * (v->rows + 1);
     out->escape_bytes = 2 * v->n_esc;
     out->escape_rate = static_cast<double>(v->n_esc) / static_cast<double>(nw);
     out->bits_per_weight = 8.0 * static_cast<double>(v->container_bytes) / static_cast<double>(nw);

@@ -118,7 +118,7 @@ typedef struct s12_stats_t {
     uint64_t rows, cols, n_tiles, n_esc;
     uint64_t container_bytes; /* everything, padding included            */
     uint64_t payload_bytes;   /* raw + code = 1.5 bytes per weight       */
-    uint64_t header_bytes;    /* 5 bytes per tile (base + offset)        */
+    uint64_t header_bytes;    /* v1: 5 per tile; v2: 2 per tile + 4 per row */
     uint64_t escape_bytes;    /* 2 bytes per escape                      */
     double escape_rate;       /* n_esc / (rows*cols)                     */
     double bits_per_weight;   /* 8 * container_bytes / (rows*cols)       */

@@ -21,6 +21,9 @@ def test_reference_arm_json_line():
     sys.path.insert(0, ROOT)
     import bench
     assert d["impl"] == "reference"
+    # the same config dict as the library arm prints, so the two lines compare
+    import bench
+    assert d["config"] == bench.llama_config(1, 1)
     assert d["metric"] == bench.METRIC and d["unit"] == "GB/s" and d["higher_is_better"] is True
     assert d["n_gpus"] == 1 and d["steps"] == 1 and d["warmup"] == 3
     assert d["value"] > 0 and d["ms_per_step"] > 0

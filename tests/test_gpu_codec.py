@@ -202,3 +202,65 @@ def test_size_query_and_capacity(s12, oracle):
     rc = lib.s12_encode(C.c_void_p(wd.data_ptr()), 8, 256, C.c_void_p(small.data_ptr()), small.numel(),
                         C.byref(n), C.c_void_p(ws.data_ptr()), ws.numel(), st)
     assert rc == s12.S12_ERR_CAPACITY
+
+
+# ---------------------------------------------------------------------------
+# container version 2 on the GPU: the decoder and the statistics read it
+
+@pytest.mark.parametrize("order", ["natural", "shuffled"])
+def test_v2_decode_all_patterns(s12, oracle, order):
+    """All 65,536 BF16 patterns as a version 2 container built by the oracle:
+    the GPU decode gives every bit back and raises no flag."""
+    w = _all_patterns(order)
+    blob = blob_to_dev(oracle.encode_v2(w))
+    view = s12.s12_open(blob)
+    assert view.version == 2
+    flag = new_flag()
+    out = s12.s12_decode(view, err_flag=flag)
+    torch.cuda.synchronize()
+    assert np.array_equal(from_dev_u16(out), w)
+    assert int(flag.item()) == 0
+
+
+@pytest.mark.parametrize("shape", [(1, 128), (3, 384), (67, 384), (300, 1152), (33, 4096), (5, 14336)])
+@pytest.mark.parametrize("rate", [0.0003, 0.10])
+def test_v2_decode_shapes_and_escape_rates(s12, oracle, shape, rate):
+    """Version 2 decode at a low and a high escape rate, over chunks that
+    cross row boundaries and ragged final chunks (n_tiles not a multiple of
+    32): bit-exact against the source matrix."""
+    r, c = shape
+    w, _ = wl.escape_stress(rate, r + c, r, c)
+    blob = blob_to_dev(oracle.encode_v2(w))
+    view = s12.s12_open(blob)
+    flag = new_flag()
+    out = s12.s12_decode(view, err_flag=flag)
+    torch.cuda.synchronize()
+    assert np.array_equal(from_dev_u16(out), w)
+    assert int(flag.item()) == 0
+
+
+def test_v2_decode_full_size_escape_stress(s12, oracle):
+    """8192 x 8192 at 2 % escapes as a version 2 container: bit-exact."""
+    w, planted = wl.escape_stress(0.02, seed=0)
+    blob = blob_to_dev(oracle.encode_v2(w))
+    view = s12.s12_open(blob)
+    assert view.n_esc == planted
+    flag = new_flag()
+    out = s12.s12_decode(view, err_flag=flag)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), to_dev(w))
+    assert int(flag.item()) == 0
+
+
+def test_v2_stats_match_v1(s12, oracle):
+    """The statistics of a version 2 container: the same exponent histogram
+    and entropy as the oracle's statistics of the version 1 container, and
+    the header bytes of version 2 (2 per tile + 4 per row)."""
+    w = wl.student_t_scaled(300, 1152, 5)
+    ref = oracle.stats(oracle.encode(w))
+    view = s12.s12_open(blob_to_dev(oracle.encode_v2(w)))
+    st = s12.s12_stats(view)
+    assert st["exp_hist"] == [int(h) for h in ref["exp_hist"]]
+    assert st["exp_entropy_bits"] == pytest.approx(ref["exp_entropy_bits"], abs=1e-12)
+    assert st["header_bytes"] == 2 * view.n_tiles + 4 * (view.rows + 1)
+    assert st["n_esc"] == ref["n_esc"]
