@@ -791,8 +791,14 @@ def mlp_swiglu_extras(layer, world, steps: int):
 
 def stack_extras(world, layers: int = 32, steps: int = 10):
     """Whole-stack weight streaming: `layers` independent 8B-style layers
-    (layer l drawn with seed l) resident as Split12 containers, one grouped
-    launch per layer (its seven GEMVs), one pass = all layers; B = 1 and 8.
+    (layer l drawn with seed l) resident as Split12 containers (gate and up
+    as one interleaved container), one pass = all layers; B = 1 and 8.
+    Two forms: one grouped launch per layer over its six containers (pure
+    weight streaming), and the activation chain, where the layer's down
+    output (BF16) is the next layer's input: per layer q, k, v, o in one
+    grouped launch (attention is outside the path: o reads the layer input
+    in its place), gate/up with the SwiGLU epilogue, down with a BF16
+    output.
     Plus an 8-expert MoE block (gate, up 14336x4096, down 4096x14336 per
     expert) with top-2 routing of 64 tokens: experts with >= 9 tokens use the
     skinny GEMM (rows padded to 16), the rest the GEMV."""
@@ -800,14 +806,23 @@ def stack_extras(world, layers: int = 32, steps: int = 10):
 
     from decode_split12_b200 import s12
     hbm, _, _, _ = load_peaks()
-    names = list(wl.LLAMA8B_SHAPES)
+    # containers per layer: q, k, v, o, gate/up interleaved, down
+    names = ["q", "k", "v", "o", "gate_up", "down"]
+    shapes = {n: wl.LLAMA8B_SHAPES[n] for n in ("q", "k", "v", "o", "down")}
+    F, Dm = wl.LLAMA8B_SHAPES["gate"]
+    shapes["gate_up"] = (2 * F, Dm)
     blobs, views = [], []
     for layer in range(layers):
         gen = torch.Generator(device="cuda").manual_seed(layer)
         lv = []
         for n in names:
-            r, c = wl.LLAMA8B_SHAPES[n]
-            wd = _student_t_gpu(r, c, gen)
+            if n == "gate_up":
+                wg = _student_t_gpu(F, Dm, gen)
+                wu = _student_t_gpu(F, Dm, gen)
+                wd = s12.interleave_gate_up(wg, wu)
+                del wg, wu
+            else:
+                wd = _student_t_gpu(*shapes[n], gen)
             b = s12.s12_encode(wd)
             del wd
             blobs.append(b)
@@ -819,8 +834,8 @@ def stack_extras(world, layers: int = 32, steps: int = 10):
     ws = torch.zeros(s12.s12_gemv_multi_ws_bytes(views[0], 8), dtype=torch.uint8, device="cuda")
     out = {"layers": layers, "weights": weights, "container_bytes": cbytes}
     for B in (1, 8):
-        xs = [dev16(wl.activations(B, wl.LLAMA8B_SHAPES[n][1], B, 3000 + i)) for i, n in enumerate(names)]
-        ys = [torch.empty((B, wl.LLAMA8B_SHAPES[n][0]), dtype=torch.float32, device="cuda") for n in names]
+        xs = [dev16(wl.activations(B, shapes[n][1], B, 3000 + i)) for i, n in enumerate(names)]
+        ys = [torch.empty((B, shapes[n][0]), dtype=torch.float32, device="cuda") for n in names]
 
         def step():
             for lv in views:
@@ -833,6 +848,31 @@ def stack_extras(world, layers: int = 32, steps: int = 10):
         out[f"B{B}"] = {"ms_per_pass": round(t * 1e3, 3), "ms_per_token": round(t * 1e3 / B, 3),
                         "effective_bf16_GBs": round(2 * weights / t / 1e9, 1),
                         "hbm_frac": round(cbytes / t / 1e9 / hbm, 4), "launches_per_pass": layers}
+        del g
+    # the activation chain (each layer's GEMVs depend on the previous layer)
+    for B in (1, 8):
+        h0 = dev16(wl.activations(B, Dm, B, 5000))
+        hs = [h0] + [torch.empty((B, Dm), dtype=torch.int16, device="cuda") for _ in range(layers)]
+        hid = torch.empty((B, F), dtype=torch.int16, device="cuda")
+        yp = [torch.empty((B, shapes[n][0]), dtype=torch.float32, device="cuda") for n in ("q", "k", "v", "o")]
+
+        def chain():
+            for l, lv in enumerate(views):
+                h = hs[l]
+                s12.s12_gemv_multi(lv[:4], [h] * 4, yp, ws=ws)
+                s12.s12_gemv_swiglu(lv[4], h, hid, ws=ws)
+                s12.s12_gemv_bf16(lv[5], hid, hs[l + 1], ws=ws)
+
+        g = capture(chain)
+        for _ in range(3):
+            g.replay()
+        t = time_graph(g, steps, world) / steps
+        last = hs[layers].view(torch.bfloat16).float()
+        out[f"chain_B{B}"] = {"ms_per_pass": round(t * 1e3, 3), "ms_per_token": round(t * 1e3 / B, 3),
+                              "effective_bf16_GBs": round(2 * weights / t / 1e9, 1),
+                              "hbm_frac": round(cbytes / t / 1e9 / hbm, 4), "launches_per_pass": 3 * layers,
+                              "output_finite": bool(torch.isfinite(last).all()),
+                              "output_rms": float(last.pow(2).mean().sqrt())}
         del g
     del blobs, views
     torch.cuda.empty_cache()

@@ -42,8 +42,19 @@
 //
 // Every wait is bounded (about a second); a wait that gives up raises
 // S12_FLAG_TIMEOUT and the CTA unwinds, waiting (bounded) for its copies in
-// flight and freeing its TMEM before it exits.
+// flight and freeing its TMEM before it exits.  An unwinding CTA still
+// arrives on the counter of every shared tile it had not yet finished, so
+// the counters return to zero (Y is then not valid; the flag says so).
+//
+// Both container versions are read: version 1 keeps per tile a base byte and
+// an escape offset; version 2 (compact header) keeps per tile one u16 of
+// base | escape count and per row one escape offset, and each decode thread
+// carries its row's running offset from tile column to tile column.  Y is
+// written as FP32 or, for callers whose next step takes BF16, rounded to
+// BF16 (nearest even).
 #include <algorithm>
+
+#include <cuda_bf16.h>
 
 #include "s12_device.cuh"
 #include "s12_launch.h"
@@ -70,11 +81,12 @@ struct __align__(64) Problem {
     CUtensorMap tm_raw;   // u8 [N][K], box 128 x 128, 128-byte swizzle
     CUtensorMap tm_code;  // u8 [N][K/2], box 64 x 128
     CUtensorMap tm_x;     // bf16 [M][K], box 64 x Mp, 128-byte swizzle (rows >= M read as 0)
-    const uint8_t *base;
-    const uint32_t *esc_off;
+    const void *meta;       // version 1: base u8[n_tiles]; version 2: (base | count << 8) u16[n_tiles]
+    const uint32_t *off;    // version 1: esc_off u32[n_tiles + 1]; version 2: row_esc u32[N + 1]
     const uint16_t *esc;
     uint64_t n_esc;
-    float *y;               // M x N fp32
+    void *y;                // M x N, fp32 (out 0) or bf16 (out 1)
+    int out;
     long long unit0;        // first unit of this matrix in the call's numbering
     int N, K, T, M;
     int n_tiles, n_chunks;  // tiles of 128 rows; 128-column units per row (= tiles per row)
@@ -231,7 +243,7 @@ namespace gemm {
 // Shared-memory layout (offsets from the 1024-aligned base).
 struct Layout {
     uint32_t full, empty, a_full, a_empty, acc_full, acc_empty, done;  // mbarriers
-    uint32_t tmem_slot, xchg;                                     // 4-byte words
+    uint32_t tmem_slot, xchg, abort, n_done;                      // 4-byte words
     uint32_t stages, abuf;                                        // data regions
 };
 
@@ -247,6 +259,8 @@ __device__ __forceinline__ Layout layout(uint32_t sb, const Params<NP> &p) {
     L.done = L.acc_empty + 8;
     L.tmem_slot = L.done + 8;
     L.xchg = L.tmem_slot + 4;
+    L.abort = L.xchg + 4;   // set when a wait of this CTA gave up
+    L.n_done = L.abort + 4; // tiles of this CTA whose counter arrival is done (or not needed)
     L.stages = sb + 1024;
     L.abuf = L.stages + static_cast<uint32_t>(p.stages) * p.stage_bytes;
     return L;
@@ -258,10 +272,29 @@ __device__ __forceinline__ Layout layout(uint32_t sb, const Params<NP> &p) {
 // Per-tile metadata of one row: base and escape offsets.
 // (Escape values are read when a unit needs them: fetching a row's first
 // two one unit ahead cost more per unit than it hid, 6 % at M = 16.)
+// The words as loaded (any arithmetic on them at load time would make the
+// thread wait for the load there):
+//   version 1:  w0 = base, w1 = esc_off[t], w2 = esc_off[t+1]
+//   version 2:  w0 = tmeta[t], w1 = row_esc[n] on a row's first tile column
 struct RowMeta {
-    uint32_t base, lo, hi;
+    uint32_t w0, w1, w2;
     int pi;  // the matrix the unit belongs to
 };
+
+// Base and escape span [lo, hi) of a row's tile; `run` carries the row's
+// escape offset (version 2) from one tile column to the next.
+struct RowSpan {
+    uint32_t base, lo, hi;
+};
+
+template <int V>
+__device__ __forceinline__ RowSpan row_span(const RowMeta &m, int chunk, uint32_t &run) {
+    if (V == 1) return RowSpan{m.w0, m.w1, m.w2};
+    if (chunk == 0) run = m.w1;
+    const RowSpan s{m.w0 & 0xFFu, run, run + (m.w0 >> 8)};
+    run = s.hi;
+    return s;
+}
 
 // Rows past the end (zeros from the copy engine) read the last row's
 // metadata but report no escapes.
@@ -298,19 +331,42 @@ __device__ __forceinline__ UPos locate(const Params<NP> &P, long long u) {
     return q;
 }
 
-template <int NP>
+template <int V, int NP>
 __device__ __forceinline__ RowMeta load_row_meta(const Params<NP> &P, UPos q, int r) {
     const Problem &p = P.prob[q.p];
     const int tile = q.tile, j = q.chunk;  // a unit is one whole tile column
     const int n = tile * kRows + r;
-    const size_t t = static_cast<size_t>(min(n, p.N - 1)) * p.T + j;
+    const int nc = min(n, p.N - 1);
+    const size_t t = static_cast<size_t>(nc) * p.T + j;
     RowMeta m;
-    m.base = __ldg(p.base + t);
-    m.lo = __ldg(p.esc_off + t);
-    m.hi = __ldg(p.esc_off + t + 1);
-    if (n >= p.N) m.hi = m.lo;
+    if (V == 1) {
+        m.w0 = __ldg(static_cast<const uint8_t *>(p.meta) + t);
+        m.w1 = __ldg(p.off + t);
+        m.w2 = n < p.N ? __ldg(p.off + t + 1) : m.w1;
+    } else {
+        const uint32_t w = __ldg(static_cast<const uint16_t *>(p.meta) + t);
+        m.w0 = n < p.N ? w : (w & 0xFFu);  // rows past the end: no escapes
+        m.w1 = j == 0 ? __ldg(p.off + nc) : 0u;
+        m.w2 = 0u;
+    }
     m.pi = q.p;
     return m;
+}
+
+// Version 2: escape offset of row r of the unit at q before its tile column
+// (row_esc plus the counts of the row's earlier tiles), summed by the four
+// lanes that share the row (lanes l, l^8, l^16, l^24; lane q4 takes tiles
+// q4, q4 + 4, ...).
+template <int NP>
+__device__ __forceinline__ uint32_t row_offset_v2(const Params<NP> &P, UPos q, int r, int q4) {
+    const Problem &p = P.prob[q.p];
+    const int nc = min(q.tile * kRows + r, p.N - 1);
+    const uint16_t *tm = static_cast<const uint16_t *>(p.meta) + static_cast<size_t>(nc) * p.T;
+    uint32_t s = 0;
+    for (int k = q4; k < q.chunk; k += 4) s += __ldg(tm + k) >> 8;
+    s += __shfl_xor_sync(0xFFFFFFFFu, s, 8);
+    s += __shfl_xor_sync(0xFFFFFFFFu, s, 16);
+    return s + __ldg(p.off + nc);
 }
 
 // Decode the lane's 32 weights of one tile row (row r of the unit, columns
@@ -320,7 +376,7 @@ __device__ __forceinline__ RowMeta load_row_meta(const Params<NP> &P, UPos q, in
 // order: lane q4 = 0..3, first chunk then second).
 template <bool CHECK>
 __device__ __forceinline__ void decode_row(const Problem &p, uint32_t *err, uint32_t st_raw, uint32_t st_code,
-                                           uint32_t abuf, int r, int q4, const RowMeta &rm) {
+                                           uint32_t abuf, int r, int q4, const RowSpan &rm) {
     const uint32_t sw = static_cast<uint32_t>(r & 7);
     const uint32_t lo = rm.lo, hi = rm.hi;
     const uint4 rw0 = lds128(st_raw + r * 128 + (((2u * q4) ^ sw) << 4));  // raw rows are 128-byte swizzled
@@ -396,6 +452,63 @@ __device__ __forceinline__ void decode_row(const Problem &p, uint32_t *err, uint
 namespace s12 {
 namespace gemm {
 
+__device__ __forceinline__ void store_y(const Problem &pr, size_t o, float v) {
+    if (pr.out == 1)
+        static_cast<uint16_t *>(pr.y)[o] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+    else
+        static_cast<float *>(pr.y)[o] = v;
+}
+
+// One more tile of this CTA has its counter arrival behind it (or needs none).
+__device__ __forceinline__ void note_done(const Layout &L) {
+    uint32_t n;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(n) : "r"(L.n_done) : "memory");
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(L.n_done), "r"(n + 1) : "memory");
+}
+
+// A wait gave up: raise the flag and mark the CTA as unwinding.
+template <int NP>
+__device__ __forceinline__ void give_up(const Params<NP> &p, const Layout &L) {
+    raise_flag(p.err, S12_FLAG_TIMEOUT);
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(L.abort), "r"(1u) : "memory");
+}
+
+// Number of CTAs whose unit range meets tile units [t0, t1).
+__device__ __forceinline__ uint32_t contributors(long long t0, long long t1, long long n_units, int grid) {
+    const long long cf = cta_of_unit(t0, n_units, grid), cl = cta_of_unit(t1 - 1, n_units, grid);
+    uint32_t n = 0;
+    for (long long c = cf; c <= cl; ++c)
+        if (unit_start(c, n_units, grid) < unit_start(c + 1, n_units, grid)) ++n;
+    return n;
+}
+
+// After an unwinding CTA's threads have all stopped: arrive on the counter of
+// every tile of its range that it shares with other CTAs and had not yet
+// finished, resetting the counter when this arrival is the last.  Run by one
+// thread.
+template <int NP>
+__device__ void abort_arrivals(const Params<NP> &p, const Layout &L, long long u0, long long u1) {
+    uint32_t n_done;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(n_done) : "r"(L.n_done) : "memory");
+    UPos q = locate(p, u0);
+    uint32_t k = 0;
+    for (long long u = u0; u < u1; ++k) {
+        const Problem &pr = p.prob[q.p];
+        const long long t0 = pr.unit0 + static_cast<long long>(q.tile) * pr.n_chunks, t1 = t0 + pr.n_chunks;
+        if (k >= n_done && !(t0 >= u0 && t1 <= u1)) {
+            const uint32_t gtile = static_cast<uint32_t>(pr.tile0 + q.tile);
+            const uint32_t prev = atomicAdd(p.cnt + gtile, 1u);
+            if (prev + 1 == contributors(t0, t1, p.n_units, gridDim.x)) atomicExch(p.cnt + gtile, 0u);
+        }
+        u = t1;
+        q.chunk = 0;
+        if (++q.tile == pr.n_tiles) {
+            q.tile = 0;
+            ++q.p;
+        }
+    }
+}
+
 // Epilogue for tile `tile` of matrix pr (the accumulators are final for this
 // CTA's part of it): store Y directly, or hand the partial to the stream-K
 // fix-up.  gtile is the tile's index in the call's numbering (its counter),
@@ -426,13 +539,16 @@ __device__ __forceinline__ void epilogue(const Params<NP> &p, const Problem &pr,
         for (int i = 0; i < 4; ++i) {
             const int m = c + i;
             if (whole) {
-                if (m < pr.M && n < pr.N) pr.y[static_cast<size_t>(m) * pr.N + n] = __uint_as_float(v[i]);
+                if (m < pr.M && n < pr.N) store_y(pr, static_cast<size_t>(m) * pr.N + n, __uint_as_float(v[i]));
             } else {
                 __stcg(mine + static_cast<size_t>(m) * kRows + row, __uint_as_float(v[i]));
             }
         }
     }
-    if (whole) return;
+    if (whole) {
+        if (ew == 0 && lane == 0) note_done(L);
+        return;
+    }
     // stream-K fix-up: the last contributor of the tile adds the partials in
     // CTA order and writes Y
     __threadfence();
@@ -441,10 +557,9 @@ __device__ __forceinline__ void epilogue(const Params<NP> &p, const Problem &pr,
     const int grid = gridDim.x;
     const long long cf = cta_of_unit(t0, n_units, grid), cl = cta_of_unit(t1 - 1, n_units, grid);
     if (ew == 0 && lane == 0) {
-        uint32_t n_contrib = 0;
-        for (long long c = cf; c <= cl; ++c)
-            if (unit_start(c, n_units, grid) < unit_start(c + 1, n_units, grid)) ++n_contrib;
+        const uint32_t n_contrib = contributors(t0, t1, n_units, grid);
         const uint32_t prev = atomicAdd(p.cnt + gtile, 1u);
+        note_done(L);
         asm volatile("st.shared.u32 [%0], %1;" ::"r"(L.xchg), "r"(prev + 1 == n_contrib ? 1u : 0u) : "memory");
     }
     asm volatile("bar.sync 1, %0;" ::"n"(32 * kDecodeWarps) : "memory");
@@ -463,13 +578,13 @@ __device__ __forceinline__ void epilogue(const Params<NP> &p, const Problem &pr,
                         static_cast<size_t>(idx));
         }
         const int nn = tile * kRows + r;
-        if (m < pr.M && nn < pr.N) pr.y[static_cast<size_t>(m) * pr.N + nn] = s;
+        if (m < pr.M && nn < pr.N) store_y(pr, static_cast<size_t>(m) * pr.N + nn, s);
     }
     asm volatile("bar.sync 1, %0;" ::"n"(32 * kDecodeWarps) : "memory");
     if (ew == 0 && lane == 0) atomicExch(p.cnt + gtile, 0u);
 }
 
-template <bool CHECK, int NP>
+template <bool CHECK, int NP, int V>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ Params<NP> p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t sb = (smem_addr(smem_raw) + 1023u) & ~1023u;
@@ -491,6 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         bar_init(L.acc_full, 1);
         bar_init(L.acc_empty, kDecodeWarps);
         bar_init(L.done, 1);
+        asm volatile("st.shared.v2.u32 [%0], {%1, %1};" ::"r"(L.abort), "r"(0u) : "memory");
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -515,7 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                 const Problem &pr = p.prob[q.p];
                 const int tile = q.tile, chunk = q.chunk;
                 if (!bar_wait(L.empty + 8 * s, (round & 1u) ^ 1u)) {
-                    raise_flag(p.err, S12_FLAG_TIMEOUT);
+                    give_up(p, L);
                     break;
                 }
                 const uint32_t st = L.stages + static_cast<uint32_t>(s) * p.stage_bytes;
@@ -549,7 +665,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                 bool w = bar_wait(L.full + 8 * s, round & 1u) && bar_wait(L.a_full + 8 * a, around & 1u);
                 if (w && first) w = bar_wait(L.acc_empty, (tiles & 1u) ^ 1u);
                 if (!w) {
-                    raise_flag(p.err, S12_FLAG_TIMEOUT);
+                    give_up(p, L);
                     break;
                 }
                 if (first) ++tiles;
@@ -588,27 +704,31 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         RowMeta m0 = {0, 0, 0, 0}, m1 = {0, 0, 0, 0};
         UPos q = q0;
         UPos qm = q;  // the unit whose metadata is loaded next
-        if (u0 < u1) m0 = load_row_meta(p, qm, r);
+        if (u0 < u1) m0 = load_row_meta<V>(p, qm, r);
         next(qm, p);
-        if (u0 + 1 < u1) m1 = load_row_meta(p, qm, r);
+        if (u0 + 1 < u1) m1 = load_row_meta<V>(p, qm, r);
         next(qm, p);
+        // version 2: the row's escape offset at the current tile column
+        uint32_t run = 0;
+        if (V == 2 && u0 < u1 && q0.chunk > 0) run = row_offset_v2(p, q0, r, q4);
         for (long long u = u0; u < u1; ++u, next(q, p)) {
             const Problem &pr = p.prob[q.p];
             const int tile = q.tile, chunk = q.chunk;
             const bool last = (u + 1 == u1) || chunk == pr.n_chunks - 1;
             RowMeta m2 = m1;
             if (u + 2 < u1) {
-                m2 = load_row_meta(p, qm, r);
+                m2 = load_row_meta<V>(p, qm, r);
                 next(qm, p);
             }
             const bool w = bar_wait(L.full + 8 * s, round & 1u) && bar_wait(L.a_empty + 8 * a, (around & 1u) ^ 1u);
             if (!__all_sync(0xFFFFFFFFu, w)) {
-                raise_flag(p.err, S12_FLAG_TIMEOUT);
+                give_up(p, L);
                 break;
             }
             const uint32_t st = L.stages + static_cast<uint32_t>(s) * p.stage_bytes;
             const uint32_t aa = L.abuf + static_cast<uint32_t>(a) * kABytes;
-            decode_row<CHECK>(pr, p.err, st + p.x_bytes, st + p.x_bytes + kRawBytes, aa, r, q4, m0);
+            decode_row<CHECK>(pr, p.err, st + p.x_bytes, st + p.x_bytes + kRawBytes, aa, r, q4,
+                              row_span<V>(m0, chunk, run));
             m0 = m1;
             m1 = m2;
             // generic-proxy stores must be visible to the tensor core
@@ -629,7 +749,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             if (last) {
                 const bool wa = bar_wait(L.acc_full, tiles & 1u);
                 if (!__all_sync(0xFFFFFFFFu, wa)) {
-                    raise_flag(p.err, S12_FLAG_TIMEOUT);
+                    give_up(p, L);
                     break;
                 }
                 ++tiles;
@@ -646,6 +766,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, p.tmem_cols);
+    }
+    if (warp == 2 && lane == 0) {
+        uint32_t ab;
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(ab) : "r"(L.abort) : "memory");
+        if (ab) abort_arrivals(p, L, u0, u1);
     }
 }
 
@@ -702,9 +827,9 @@ Plan plan(const s12_view *views, int count, const int *M, int sms) {
     return pl;
 }
 
-template <bool CHECK, int NP>
-int run_gemm(const s12_view *views, int count, const uint16_t *const *x, const int *M, float *const *y, void *ws,
-             uint32_t *err, const Plan &pl, cudaStream_t stream) {
+template <bool CHECK, int NP, int V>
+int run_gemm(const s12_view *views, int count, const uint16_t *const *x, const int *M, void *const *y,
+             const int *out, void *ws, uint32_t *err, const Plan &pl, cudaStream_t stream) {
     gemm::Params<NP> p = {};
     long long unit0 = 0;
     int tile0 = 0;
@@ -719,11 +844,12 @@ int run_gemm(const s12_view *views, int count, const uint16_t *const *x, const i
         if (make_tmap_bf16_2d(&q.tm_x, x[i], K, static_cast<uint64_t>(M[i]), K * 2, gemm::kAtom,
                               static_cast<uint32_t>(pl.Mp), 128) != S12_OK)
             return S12_ERR_CUDA;
-        q.base = v->base;
-        q.esc_off = v->esc_off;
+        q.meta = V == 1 ? static_cast<const void *>(v->base) : static_cast<const void *>(v->tmeta);
+        q.off = V == 1 ? v->esc_off : v->row_esc;
         q.esc = v->esc;
         q.n_esc = v->n_esc;
         q.y = y[i];
+        q.out = out ? out[i] : 0;
         q.N = static_cast<int>(N);
         q.K = static_cast<int>(K);
         q.T = q.K / kTile;
@@ -747,7 +873,7 @@ int run_gemm(const s12_view *views, int count, const uint16_t *const *x, const i
     p.x_atom = pl.x_atom;
     p.a_bufs = pl.a_bufs;
     p.tmem_cols = pl.tmem_cols;
-    auto kern = gemm::gemm_tc_kernel<CHECK, NP>;
+    auto kern = gemm::gemm_tc_kernel<CHECK, NP, V>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem) != cudaSuccess)
         return S12_ERR_CUDA;
     kern<<<pl.grid, gemm::kThreads, pl.smem, stream>>>(p);
@@ -763,21 +889,33 @@ size_t gemm_ws_bytes(const s12_view *views, int count, const int *M) {
     return pl.part_bytes + pl.cnt_bytes;
 }
 
-int launch_gemm(const s12_view *views, int count, const uint16_t *const *x, const int *M, float *const *y, void *ws,
-                size_t ws_bytes, uint32_t *err, cudaStream_t stream) {
-    for (int i = 0; i < count; ++i)
-        if (views[i].version != 1) return S12_ERR_ARG;
+int launch_gemm(const s12_view *views, int count, const uint16_t *const *x, const int *M, void *const *y,
+                const int *out, void *ws, size_t ws_bytes, uint32_t *err, cudaStream_t stream) {
+    // one container version per call
+    const uint32_t version = views[0].version;
+    for (int i = 0; i < count; ++i) {
+        if (views[i].version != version || (version != 1 && version != 2)) return S12_ERR_ARG;
+        if (out && out[i] != 0 && out[i] != 1) return S12_ERR_ARG;
+    }
     int sms = 0;
     if (device_sms(&sms) != cudaSuccess) return S12_ERR_CUDA;
     const Plan pl = plan(views, count, M, sms);
     if (!ws || ws_bytes < pl.part_bytes + pl.cnt_bytes) return S12_ERR_CAPACITY;
     if (pl.stages < 2) return S12_ERR_SHAPE;
     // a one-matrix call takes the small parameter block
+    constexpr int kG = gemm::kMaxProblems;
+    if (version == 1) {
+        if (count == 1)
+            return err ? run_gemm<true, 1, 1>(views, count, x, M, y, out, ws, err, pl, stream)
+                       : run_gemm<false, 1, 1>(views, count, x, M, y, out, ws, err, pl, stream);
+        return err ? run_gemm<true, kG, 1>(views, count, x, M, y, out, ws, err, pl, stream)
+                   : run_gemm<false, kG, 1>(views, count, x, M, y, out, ws, err, pl, stream);
+    }
     if (count == 1)
-        return err ? run_gemm<true, 1>(views, count, x, M, y, ws, err, pl, stream)
-                   : run_gemm<false, 1>(views, count, x, M, y, ws, err, pl, stream);
-    return err ? run_gemm<true, gemm::kMaxProblems>(views, count, x, M, y, ws, err, pl, stream)
-               : run_gemm<false, gemm::kMaxProblems>(views, count, x, M, y, ws, err, pl, stream);
+        return err ? run_gemm<true, 1, 2>(views, count, x, M, y, out, ws, err, pl, stream)
+                   : run_gemm<false, 1, 2>(views, count, x, M, y, out, ws, err, pl, stream);
+    return err ? run_gemm<true, kG, 2>(views, count, x, M, y, out, ws, err, pl, stream)
+               : run_gemm<false, kG, 2>(views, count, x, M, y, out, ws, err, pl, stream);
 }
 
 }  // namespace s12

@@ -332,8 +332,9 @@ namespace {
 // Shared checks of the GEMM calls: every entry valid, before any launch.
 // min_m: the smallest token count an entry may have (a grouped call pads
 // every matrix to the shared multiple of 16, so it accepts any M >= 1).
-int check_gemm_group(const s12_view *views, int count, const uint16_t *const *x, const int *M, float *const *y,
-                     int min_m) {
+// out: null (all FP32) or one output kind per entry (0 FP32, 1 BF16).
+int check_gemm_group(const s12_view *views, int count, const uint16_t *const *x, const int *M, void *const *y,
+                     const int *out, int min_m) {
     if (!views || !x || !M || !y || count < 1 || count > S12_GEMM_MAX_PROBLEMS) return S12_ERR_ARG;
     for (int i = 0; i < count; ++i) {
         const int rc = check_view(views + i);
@@ -341,22 +342,37 @@ int check_gemm_group(const s12_view *views, int count, const uint16_t *const *x,
         if (!x[i] || !y[i]) return S12_ERR_ARG;
         if (M[i] < min_m || M[i] > S12_GEMM_MAX_M) return S12_ERR_SHAPE;
         if (views[i].rows > 0x7FFFFFFFull || views[i].cols > 0x7FFFFFFFull) return S12_ERR_SHAPE;
-        if (!aligned16(x[i]) || !aligned4(y[i])) return S12_ERR_ALIGN;
+        const bool bf16 = out && out[i] == 1;
+        const bool y_ok = bf16 ? (reinterpret_cast<uintptr_t>(y[i]) & 1) == 0 : aligned4(y[i]);
+        if (!aligned16(x[i]) || !y_ok) return S12_ERR_ALIGN;
     }
     return S12_OK;
+}
+
+// One fused GEMM with output kind `kind` (0 FP32, 1 BF16).
+int gemm_one(const s12_view *v, const uint16_t *x, int M, void *y, int kind, void *ws, size_t ws_bytes,
+             uint32_t *err_flag, void *stream) {
+    int rc = check_view(v);
+    if (rc != S12_OK) return rc;
+    if (!x || !y) return S12_ERR_ARG;
+    void *yy[1] = {y};
+    const int out[1] = {kind};
+    rc = check_gemm_group(v, 1, &x, &M, yy, out, S12_GEMM_MIN_M);
+    if (rc != S12_OK) return rc;
+    if ((ws && !aligned16(ws)) || (err_flag && !aligned4(err_flag))) return S12_ERR_ALIGN;
+    if (ws_bytes < gemm_ws_bytes(v, 1, &M)) return S12_ERR_CAPACITY;
+    return launch_gemm(v, 1, &x, &M, yy, out, ws, ws_bytes, err_flag, static_cast<cudaStream_t>(stream));
 }
 }  // namespace
 
 int s12_gemm_skinny(const s12_view *v, const uint16_t *x, int M, float *y, void *ws, size_t ws_bytes,
                     uint32_t *err_flag, void *stream) {
-    int rc = check_view(v);
-    if (rc != S12_OK) return rc;
-    if (!x || !y) return S12_ERR_ARG;
-    rc = check_gemm_group(v, 1, &x, &M, &y, S12_GEMM_MIN_M);
-    if (rc != S12_OK) return rc;
-    if ((ws && !aligned16(ws)) || (err_flag && !aligned4(err_flag))) return S12_ERR_ALIGN;
-    if (ws_bytes < gemm_ws_bytes(v, 1, &M)) return S12_ERR_CAPACITY;
-    return launch_gemm(v, 1, &x, &M, &y, ws, ws_bytes, err_flag, static_cast<cudaStream_t>(stream));
+    return gemm_one(v, x, M, y, 0, ws, ws_bytes, err_flag, stream);
+}
+
+int s12_gemm_skinny_bf16(const s12_view *v, const uint16_t *x, int M, uint16_t *y, void *ws, size_t ws_bytes,
+                         uint32_t *err_flag, void *stream) {
+    return gemm_one(v, x, M, y, 1, ws, ws_bytes, err_flag, stream);
 }
 
 size_t s12_gemm_multi_ws_bytes(const s12_view *views, int count, const int *M) {
@@ -368,12 +384,15 @@ size_t s12_gemm_multi_ws_bytes(const s12_view *views, int count, const int *M) {
 
 int s12_gemm_skinny_multi(const s12_view *views, int count, const uint16_t *const *x, const int *M,
                           float *const *y, void *ws, size_t ws_bytes, uint32_t *err_flag, void *stream) {
-    const int rc = check_gemm_group(views, count, x, M, y, 1);
+    if (!y) return S12_ERR_ARG;
+    void *yy[S12_GEMM_MAX_PROBLEMS];
+    for (int i = 0; i < count && i < S12_GEMM_MAX_PROBLEMS; ++i) yy[i] = y[i];
+    const int rc = check_gemm_group(views, count, x, M, yy, nullptr, 1);
     if (rc != S12_OK) return rc;
     if (!ws) return S12_ERR_ARG;
     if (!aligned16(ws) || (err_flag && !aligned4(err_flag))) return S12_ERR_ALIGN;
     if (ws_bytes < gemm_ws_bytes(views, count, M)) return S12_ERR_CAPACITY;
-    return launch_gemm(views, count, x, M, y, ws, ws_bytes, err_flag, static_cast<cudaStream_t>(stream));
+    return launch_gemm(views, count, x, M, yy, nullptr, ws, ws_bytes, err_flag, static_cast<cudaStream_t>(stream));
 }
 
 size_t s12_stats_ws_bytes(void) { return 256 * sizeof(unsigned long long); }

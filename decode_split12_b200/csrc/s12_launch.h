@@ -69,7 +69,9 @@ int launch_encode(const uint16_t *w, int64_t rows, int64_t cols, void *dst, size
                   void *ws, size_t ws_bytes, cudaStream_t stream);
 int launch_stats_hist(const s12_view *v, unsigned long long *hist_dev, cudaStream_t stream);
 size_t gemm_ws_bytes(const s12_view *views, int count, const int *M);
-int launch_gemm(const s12_view *views, int count, const uint16_t *const *x, const int *M, float *const *y, void *ws,
-                size_t ws_bytes, uint32_t *err, cudaStream_t stream);
+// y[i]: float* (M[i] x rows) for out[i] == 0 (or a null `out`), uint16_t*
+// BF16 for out[i] == 1.
+int launch_gemm(const s12_view *views, int count, const uint16_t *const *x, const int *M, void *const *y,
+                const int *out, void *ws, size_t ws_bytes, uint32_t *err, cudaStream_t stream);
 
 }  // namespace s12

@@ -137,8 +137,9 @@ extern "C" int s12_plane_hashes_host(const void *container, size_t bytes, uint64
 // and per row one u32 escape offset, instead of a u8 base and a u32 offset
 // per tile: 2 bytes per tile + 4 per row instead of 5 per tile, toward the
 // 24.967 % payload reduction of "Lossless LLM Weight Compression vs 8-bit
-// GGUF" (English edition, opening summary).  The kernels read version 1;
-// these calls convert in host memory, for storage or transfer.
+// GGUF" (English edition, opening summary).  The kernels read both
+// versions; these calls convert between them in host memory, for storage or
+// transfer.
 
 namespace s12 {
 namespace {

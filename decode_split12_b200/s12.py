@@ -36,9 +36,10 @@ S12_FLAG_TIMEOUT = 8
 EXPORTED = (
     "s12_error_string", "s12_device_check", "s12_container_bytes", "s12_encode_ws_bytes", "s12_encode",
     "s12_open", "s12_decode", "s12_gemv_ws_bytes", "s12_gemv", "s12_gemv_multi_ws_bytes", "s12_gemv_multi",
-    "s12_gemv_noalloc", "s12_gemv_swiglu", "s12_gemv_bf16", "s12_gemm_ws_bytes", "s12_gemm_skinny", "s12_gemm_multi_ws_bytes",
+    "s12_gemv_noalloc", "s12_gemv_swiglu", "s12_gemv_bf16", "s12_gemm_ws_bytes", "s12_gemm_skinny",
+    "s12_gemm_skinny_bf16", "s12_gemm_multi_ws_bytes",
     "s12_gemm_skinny_multi", "s12_validate_host", "s12_plane_hashes_host", "s12_fnv1a64",
-    "s12_to_v2_host", "s12_from_v2_host", "s12_stats_ws_bytes",
+    "s12_to_v2_host", "s12_from_v2_host", "s12_load_bf16", "s12_stats_ws_bytes",
     "s12_stats", "s12_bf16_gemv",
 )
 
@@ -114,6 +115,8 @@ def _lib() -> C.CDLL:
         lib.s12_gemm_ws_bytes.restype = _SZ
         lib.s12_gemm_skinny.argtypes = [C.POINTER(View), _P, C.c_int, _P, _P, _SZ, _P, _P]
         lib.s12_gemm_skinny.restype = C.c_int
+        lib.s12_gemm_skinny_bf16.argtypes = [C.POINTER(View), _P, C.c_int, _P, _P, _SZ, _P, _P]
+        lib.s12_gemm_skinny_bf16.restype = C.c_int
         lib.s12_validate_host.argtypes = [_P, _SZ, C.POINTER(Report)]
         lib.s12_validate_host.restype = C.c_int
         lib.s12_plane_hashes_host.argtypes = [_P, _SZ, C.POINTER(C.c_uint64)]
@@ -121,6 +124,9 @@ def _lib() -> C.CDLL:
         for fn in ("s12_to_v2_host", "s12_from_v2_host"):
             getattr(lib, fn).argtypes = [_P, _SZ, _P, _SZ, C.POINTER(_SZ)]
             getattr(lib, fn).restype = C.c_int
+        lib.s12_load_bf16.argtypes = [_P, _SZ, _P, _P, C.c_uint64, C.c_uint64, _P, _SZ, _P, _P,
+                                      C.POINTER(LoadResult), _P]
+        lib.s12_load_bf16.restype = C.c_int
         lib.s12_fnv1a64.argtypes = [_P, _SZ]
         lib.s12_fnv1a64.restype = C.c_uint64
         lib.s12_gemm_multi_ws_bytes.argtypes = [C.POINTER(View), C.c_int, C.POINTER(C.c_int)]
@@ -376,6 +382,22 @@ def s12_gemm_skinny(view: View, x: torch.Tensor, y: torch.Tensor | None = None, 
     return y
 
 
+def s12_gemm_skinny_bf16(view: View, x: torch.Tensor, y: torch.Tensor | None = None,
+                         ws: torch.Tensor | None = None, err_flag: torch.Tensor | None = None,
+                         stream=None) -> torch.Tensor:
+    """s12_gemm_skinny with the result rounded to BF16 (returned as int16 bits)."""
+    x = _u16(x)
+    M = x.shape[0]
+    if y is None:
+        y = torch.empty((M, view.rows), dtype=torch.int16, device=x.device)
+    need = s12_gemm_ws_bytes(view, M)
+    if ws is None:
+        ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=x.device)
+    _check(_lib().s12_gemm_skinny_bf16(C.byref(view), _dptr(x), M, _dptr(y), _dptr(ws), ws.numel(),
+                                       _dptr(err_flag), _stream(stream)), "s12_gemm_skinny_bf16")
+    return y
+
+
 def s12_stats(view: View, ws: torch.Tensor | None = None, stream=None) -> dict:
     lib_ = _lib()
     if ws is None:
@@ -467,6 +489,46 @@ def _convert(fn_name: str, container) -> np.ndarray:
     out = np.zeros(n.value, np.uint8)
     _check(fn(b.ctypes.data_as(C.c_void_p), b.size, out.ctypes.data_as(C.c_void_p), out.size, C.byref(n)), fn_name)
     return out
+
+
+class LoadResult(C.Structure):
+    _fields_ = [("outcome", C.c_uint32), ("problem", C.c_uint32), ("hash_mismatch", C.c_uint32),
+                ("device_flags", C.c_uint32)]
+
+
+LOAD_OUTCOMES = {0: "decoded", 1: "fallback", 2: "rejected"}
+
+
+def s12_load_bf16(container, rows: int, cols: int, dev_container, dev_out, dev_err, expected_hashes=None,
+                  fallback=None, stream=None) -> dict:
+    """Whole-tensor load with fallback (argument marshalling for the C call).
+    container: host container bytes; expected_hashes: 5 ints or None;
+    fallback: host uint16 array (rows x cols) or None; dev_container,
+    dev_out (rows x cols 16-bit) and dev_err (one 32-bit word): device
+    tensors, or plain integer addresses (a rejection never touches them).
+    Returns the outcome ("decoded", "fallback" or "rejected") and the
+    checks' findings."""
+    b = _host_bytes(container)
+    hashes = (C.c_uint64 * 5)(*expected_hashes) if expected_hashes is not None else None
+    fb = None
+    if fallback is not None:
+        fb = np.ascontiguousarray(np.asarray(fallback).view(np.uint16))
+        if fb.size != rows * cols:
+            raise ValueError("fallback must hold rows x cols values")
+
+    def addr(t):
+        return t if isinstance(t, int) else _dptr(t)
+
+    # an address given as an integer is taken to have room for the container
+    cap_bytes = b.size if isinstance(dev_container, int) else dev_container.numel() * dev_container.element_size()
+    st = _stream(stream) if (stream is not None or torch.cuda.is_available()) else None
+    res = LoadResult()
+    _check(_lib().s12_load_bf16(b.ctypes.data_as(C.c_void_p), b.size, hashes,
+                                fb.ctypes.data_as(C.c_void_p) if fb is not None else None, rows, cols,
+                                addr(dev_container), cap_bytes, addr(dev_out), addr(dev_err), C.byref(res), st),
+           "s12_load_bf16")
+    return {"outcome": LOAD_OUTCOMES[res.outcome], "problem": S12_BAD_NAMES.get(res.problem),
+            "hash_mismatch": int(res.hash_mismatch), "device_flags": int(res.device_flags)}
 
 
 def to_v2_host(container) -> np.ndarray:

@@ -203,7 +203,8 @@ size_t s12_gemv_ws_bytes(const s12_view *v, int B);
  *   ws: device workspace of at least s12_gemv_ws_bytes(v, B) bytes (else
  *       S12_ERR_CAPACITY), owned by the caller.  It must be ZERO-FILLED
  *       before its first use (for instance one cudaMemsetAsync after
- *       allocation); every call leaves it zero-filled again when it returns.
+ *       allocation); every call leaves it zero-filled again when it returns,
+ *       a call whose bounded waits gave up (S12_FLAG_TIMEOUT) included.
  *       Two calls that may run at the same time (different streams) need
  *       different workspaces.
  * Each warp decodes 16 rows x 128 columns at a time into the registers of
@@ -311,11 +312,22 @@ size_t s12_gemm_ws_bytes(const s12_view *v, int M);
  * y[m][n] = sum_k W[n][k] * x[m][k] for 16 <= M <= 256.
  *   x: device BF16, M x cols row-major.  y: device FP32, M x rows row-major,
  *   overwritten.  ws: device scratch of s12_gemm_ws_bytes(v, M) bytes,
- *   ZERO-FILLED before its first use; every call leaves it zero-filled.
+ *   ZERO-FILLED before its first use; every call leaves it zero-filled,
+ *   a call whose bounded waits gave up (S12_FLAG_TIMEOUT) included.
  * Decoded BF16 tiles are written to shared memory and multiplied by the
- * tensor cores with FP32 accumulation. */
+ * tensor cores with FP32 accumulation.  Reads container version 1 or 2. */
 int s12_gemm_skinny(const s12_view *v, const uint16_t *x, int M, float *y, void *ws,
                     size_t ws_bytes, uint32_t *err_flag, void *stream);
+
+/* Follows: as s12_gemm_skinny ([W] "How does this compare with prior
+ * lossless systems?": fused decompression-GEMM); the BF16 result is this
+ * library's own option for callers whose next step takes BF16.
+ * s12_gemm_skinny with a BF16 output: y[m][n] = bf16_rne(FP32 sum).
+ *   y: device BF16, M x rows row-major (2-byte alignment), overwritten.
+ * The rounding adds up to 2^-9 |y| to the error of the FP32 sum.  Other
+ * arguments, errors and the workspace as for s12_gemm_skinny. */
+int s12_gemm_skinny_bf16(const s12_view *v, const uint16_t *x, int M, uint16_t *y, void *ws,
+                         size_t ws_bytes, uint32_t *err_flag, void *stream);
 
 /* Workspace bytes s12_gemm_skinny_multi needs for these `count` containers
  * with token rows M[i] (0 for invalid arguments). */
@@ -342,7 +354,8 @@ size_t s12_gemm_multi_ws_bytes(const s12_view *views, int count, const int *M);
  * a matrix's own M are read as zeros and never stored), so matrices of
  * similar M group best.  Each y[i] equals what s12_gemm_skinny gives for
  * that matrix up to the summation order, within the same tolerance.  A bad
- * entry fails the whole call before any launch. */
+ * entry fails the whole call before any launch; so does a call that mixes
+ * container versions. */
 int s12_gemm_skinny_multi(const s12_view *views, int count, const uint16_t *const *x, const int *M,
                           float *const *y, void *ws, size_t ws_bytes, uint32_t *err_flag, void *stream);
 
@@ -401,6 +414,46 @@ int s12_plane_hashes_host(const void *container, size_t bytes, uint64_t out[5]);
  * prime 0x100000001b3), the function s12_plane_hashes_host uses. */
 uint64_t s12_fnv1a64(const void *data, size_t bytes);
 
+/* Outcome of s12_load_bf16. */
+#define S12_LOAD_DECODED 0  /* every check passed; out holds the decoded tensor    */
+#define S12_LOAD_FALLBACK 1 /* a check failed; out holds the caller's BF16 copy    */
+#define S12_LOAD_REJECTED 2 /* a check failed and no BF16 copy was given          */
+
+typedef struct s12_load_result {
+    uint32_t outcome;       /* S12_LOAD_*                                          */
+    uint32_t problem;       /* S12_BAD_* of the host validation, 0 if it passed    */
+    uint32_t hash_mismatch; /* bit i: plane i's hash differs from expected[i]      */
+    uint32_t device_flags;  /* S12_FLAG_* bits of the device decode (0 if not run) */
+} s12_load_result;
+
+/* Follows: [W] "A 14-day production-readiness pilot" (operations and
+ * reversibility: keep the original BF16 weights, check what was loaded, and
+ * fall back to the original for a tensor that fails).
+ * Load one tensor to the device as BF16, whole, with a fallback.  Steps:
+ *   1. s12_validate_host(container) and, when expected_hashes (5 values of
+ *      s12_plane_hashes_host taken at encode time) is given, the plane
+ *      hashes; the header must also say rows x cols;
+ *   2. if they pass: copy the container to dev_container, decode it into
+ *      dev_out with the device err word dev_err (cleared first), read the
+ *      word back;
+ *   3. if any check failed: with `fallback` (host BF16, rows x cols) copy it
+ *      to dev_out (outcome S12_LOAD_FALLBACK); without it leave the decision
+ *      to the caller (outcome S12_LOAD_REJECTED, dev_out not valid; the
+ *      caller may reload the tensor).
+ *   container:      host, `bytes` long, version 1 (convert a version 2 one
+ *                   with s12_from_v2_host first).
+ *   dev_container:  device, 256-byte aligned, dev_cap >= bytes (else
+ *                   S12_ERR_CAPACITY); receives the container.
+ *   dev_out:        device BF16, rows x cols.   dev_err: device u32.
+ *   res:            host, filled on S12_OK.
+ * Returns S12_OK when an outcome was reached (see res->outcome); argument,
+ * alignment and CUDA errors as usual.  SYNCHRONISES `stream`.  Steps 1 and
+ * a rejection run on the host alone. */
+int s12_load_bf16(const void *container, size_t bytes, const uint64_t *expected_hashes,
+                  const uint16_t *fallback, uint64_t rows, uint64_t cols, void *dev_container,
+                  size_t dev_cap, uint16_t *dev_out, uint32_t *dev_err, s12_load_result *res,
+                  void *stream);
+
 /* Follows: [W] English edition, opening summary (the 24.967 % payload
  * reduction leaves little room for per-tile metadata).
  * Container version 2, a compact tile header, as a storage format: the same
@@ -408,8 +461,9 @@ uint64_t s12_fnv1a64(const void *data, size_t bytes);
  * << 8) and per row one u32 escape offset instead of a u8 base and a u32
  * offset per tile (2 bytes per tile + 4 per row instead of 5 per tile; [W]
  * English edition, opening summary: the 24.967 % payload reduction leaves
- * little room for metadata).  Header as version 1 with version = 2.  The
- * kernels read version 1; these calls convert in HOST memory, snprintf-style
+ * little room for metadata).  Header as version 1 with version = 2.  Every
+ * kernel call (decode, stats, GEMV, GEMM) reads either version in device
+ * memory; these calls convert between them in HOST memory, snprintf-style
  * (dst == NULL: only *bytes_out), S12_ERR_CAPACITY if dst_cap is too small,
  * S12_ERR_CORRUPT for an invalid source (a version 1 source must pass
  * s12_validate_host; a version 2 source must have row offsets and tile

@@ -181,3 +181,91 @@ def test_gemm_multi_rejects_bad_groups(s12):
         s12.s12_gemm_skinny_multi([v] * 17, [x] * 17)
     with pytest.raises(s12.S12Error):
         s12.s12_gemm_skinny_multi([v, v], [x, to_dev(wl.activations(257, 256, 0))])
+
+
+# ---------------------------------------------------------------------------
+# container version 2 (compact tile header) and the BF16 output
+
+def _v2_blob(oracle, w):
+    """A version 2 container built by the oracle from W, on the device."""
+    from gpu_util import blob_to_dev
+    return blob_to_dev(oracle.encode_v2(w))
+
+
+@pytest.mark.parametrize("checked", [True, False])
+@pytest.mark.parametrize("shape,M", [((128, 128), 16), ((300, 1152), 17), ((1000, 4096), 64),
+                                     ((130, 14336), 48), ((640, 1024), 200), ((512, 2048), 256)])
+def test_gemm_v2_small_shapes(s12, oracle, shape, M, checked):
+    """The fused GEMM reading a version 2 container (per tile one u16 of
+    base | escape count, per row one u32 escape offset; [W] English
+    edition, opening summary) matches the FP64 oracle.  CTAs whose range
+    starts in the middle of a tile row sum the earlier tiles' counts; the
+    stream-K split tiles and ragged last tiles are covered."""
+    r, c = shape
+    w = wl.normal_with_outliers(r, c, 0.02, 0.004, r + 3 * c + M)
+    x = wl.activations(M, c, M + 2)
+    view = s12.s12_open(_v2_blob(oracle, w))
+    assert view.version == 2
+    flag = new_flag() if checked else None
+    y = s12.s12_gemm_skinny(view, to_dev(x), err_flag=flag)
+    torch.cuda.synchronize()
+    yr, sr = oracle.gemv_f64(oracle.encode(w), x)
+    assert_within_tolerance(y.cpu().numpy(), yr, sr)
+    if checked:
+        assert int(flag.item()) == 0
+
+
+def test_gemm_v2_escape_heavy_and_multi(s12, oracle):
+    """Version 2 at 10 % escapes (every tile, a row of random exponents)
+    grouped with a second version 2 matrix; a call that mixes container
+    versions is refused before any launch."""
+    w0, _ = wl.escape_stress(0.10, 3, 256, 2048)
+    g = wl.rng_for(6, 0)
+    e = g.integers(0, 161, size=2048)
+    w0[5] = ((g.integers(0, 2, 2048) << 15) | (e << 7) | g.integers(0, 128, 2048)).astype(np.uint16)
+    w1 = wl.student_t_scaled(300, 1152, 4)
+    x0, x1 = wl.activations(32, 2048, 7), wl.activations(20, 1152, 8)
+    v0, v1 = s12.s12_open(_v2_blob(oracle, w0)), s12.s12_open(_v2_blob(oracle, w1))
+    flag = new_flag()
+    ys = s12.s12_gemm_skinny_multi([v0, v1], [to_dev(x0), to_dev(x1)], err_flag=flag)
+    torch.cuda.synchronize()
+    for w, x, y in ((w0, x0, ys[0]), (w1, x1, ys[1])):
+        yr, sr = oracle.gemv_f64(oracle.encode(w), x)
+        assert_within_tolerance(y.cpu().numpy(), yr, sr)
+    assert int(flag.item()) == 0
+    v_one = s12.s12_open(s12.s12_encode(to_dev(w1)))
+    with pytest.raises(s12.S12Error):
+        s12.s12_gemm_skinny_multi([v0, v_one], [to_dev(x0), to_dev(x1)])
+
+
+def test_gemm_v2_70b_down_full_size_sampled(s12, oracle):
+    """The 70B-style down projection (8192 x 28672) as a version 2 container
+    at M = 16, 48 sampled rows against the FP64 oracle."""
+    w = wl.mlp70b("down", 0)
+    x = wl.activations(16, w.shape[1], 16)
+    view = s12.s12_open(_v2_blob(oracle, w))
+    y = s12.s12_gemm_skinny(view, to_dev(x))
+    torch.cuda.synchronize()
+    rows = np.unique(np.concatenate([[0, w.shape[0] - 1], wl.rng_for(10, 1).choice(w.shape[0], 46, replace=False)]))
+    yr, sr = oracle.gemv_f64(oracle.encode(w[rows]), x)
+    assert_within_tolerance(y.cpu().numpy()[:, rows], yr, sr)
+
+
+@pytest.mark.parametrize("shape,M", [((128, 256), 16), ((300, 1152), 33), ((1024, 4096), 128), ((640, 2048), 256)])
+def test_gemm_bf16_output(s12, oracle, shape, M):
+    """The BF16-output GEMM: each y is the FP32 sum rounded to BF16, within
+    1e-3 * sum|W x| + 2^-9 |y_ref| of the FP64 oracle (rounding to BF16 adds
+    at most half an ulp, 2^-9 relative); stream-K split tiles included."""
+    r, c = shape
+    w = wl.normal_with_outliers(r, c, 0.02, 0.002, r + c + M)
+    x = wl.activations(M, c, 60 + M)
+    view = s12.s12_open(s12.s12_encode(to_dev(w)))
+    flag = new_flag()
+    yb = s12.s12_gemm_skinny_bf16(view, to_dev(x), err_flag=flag)
+    torch.cuda.synchronize()
+    y = wl.bf16_bits_to_f32(yb.cpu().numpy().view(np.uint16)).astype(np.float64)
+    yr, sr = oracle.gemv_f64(oracle.encode(w), x)
+    err = np.abs(y - yr)
+    bound = 1e-3 * sr + 2.0 ** -9 * np.abs(yr)
+    assert (err <= bound).all(), float((err / np.maximum(bound, 1e-300)).max())
+    assert int(flag.item()) == 0
