@@ -505,9 +505,9 @@ def v2_layer(layer, world, steps: int):
 
 
 def encode_llama(layer, world):
-    """The encoder (s12_encode: size query, one synchronisation, packing) on
-    the seven matrices of the layer, timed with CUDA events around each whole
-    call.  Algorithmic bytes: read the BF16 matrix once (2 B/weight), write
+    """The encoder (s12_encode: tile windows and escape counts, one
+    synchronisation, packing; one library call per matrix) on the seven
+    matrices of the layer, timed with CUDA events around each whole call.  Algorithmic bytes: read the BF16 matrix once (2 B/weight), write
     the container (1.5 B/weight + 5 B/tile + 2 B/escape + the header)."""
     import torch
 
@@ -535,8 +535,8 @@ def encode_llama(layer, world):
         del blob
     return {"ms_layer": round(total_t * 1e3, 3), "GBs": round(total_b / total_t / 1e9, 1),
             "hbm_frac": round(total_b / total_t / 1e9 / hbm, 4), "weights": weights,
-            "timing": "CUDA events around each whole s12_encode call (size query, host sync, packing), "
-                      "best of 3 per matrix"}
+            "timing": "CUDA events around each whole s12_encode call (windows and counts, host sync, "
+                      "packing), best of 3 per matrix"}
 
 
 def run_llama8b(args, world, rank):

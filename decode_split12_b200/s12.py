@@ -212,7 +212,10 @@ def s12_container_bytes(rows: int, cols: int, n_esc: int) -> int:
 
 def s12_encode(w: torch.Tensor, ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """Encode a (rows, cols) BF16 CUDA tensor; returns the container as a
-    uint8 CUDA tensor (two library calls: size query, then encode)."""
+    uint8 CUDA tensor of exactly its size.  One library call with room for
+    escapes of up to 1/256 of the weights (a view of the first bytes is
+    returned); a matrix with more escapes takes a second call at the exact
+    size the first one reported."""
     w = _u16(w)
     rows, cols = w.shape
     lib_ = _lib()
@@ -221,12 +224,16 @@ def s12_encode(w: torch.Tensor, ws: torch.Tensor | None = None, stream=None) -> 
         ws = torch.empty(max(need_ws, 256), dtype=torch.uint8, device=w.device)
     st = _stream(stream)
     nbytes = _SZ(0)
-    _check(lib_.s12_encode(_dptr(w), rows, cols, None, 0, C.byref(nbytes), _dptr(ws), ws.numel(), st),
-           "s12_encode(size)")
-    blob = torch.empty(nbytes.value, dtype=torch.uint8, device=w.device)
-    _check(lib_.s12_encode(_dptr(w), rows, cols, _dptr(blob), blob.numel(), C.byref(nbytes), _dptr(ws),
-                           ws.numel(), st), "s12_encode")
-    return blob
+    guess = int(lib_.s12_container_bytes(rows, cols, max(1024, rows * cols // 256)))
+    blob = torch.empty(guess, dtype=torch.uint8, device=w.device)
+    rc = lib_.s12_encode(_dptr(w), rows, cols, _dptr(blob), blob.numel(), C.byref(nbytes), _dptr(ws), ws.numel(),
+                         st)
+    if rc == S12_ERR_CAPACITY and nbytes.value > guess:
+        blob = torch.empty(nbytes.value, dtype=torch.uint8, device=w.device)
+        rc = lib_.s12_encode(_dptr(w), rows, cols, _dptr(blob), blob.numel(), C.byref(nbytes), _dptr(ws),
+                             ws.numel(), st)
+    _check(rc, "s12_encode")
+    return blob[:nbytes.value]
 
 
 def s12_open(blob: torch.Tensor) -> View:

@@ -157,10 +157,13 @@ size_t s12_encode_ws_bytes(int64_t rows, int64_t cols);
  *   dst == NULL: only computes *bytes_out (the exact container size).
  *   dst != NULL: writes the whole container (header, planes, zero padding)
  *                to dst (device, dst_cap bytes); S12_ERR_CAPACITY when
- *                dst_cap < the size.
+ *                dst_cap < the size, with *bytes_out set to the size.
  * Both forms run the per-tile histogram/window and escape-count kernels and
  * then SYNCHRONISE `stream` once to read the escape total; the packing
- * kernels of the second form are then enqueued asynchronously.
+ * kernels of the second form are then enqueued asynchronously.  A caller
+ * that sizes dst for an escape count it expects (s12_container_bytes) gets
+ * the container from one call, reading W twice in all; the size query is
+ * only needed when that guess fails.
  * The result is byte-for-byte the same container on every call. */
 int s12_encode(const uint16_t *w, int64_t rows, int64_t cols, void *dst, size_t dst_cap,
                size_t *bytes_out, void *ws, size_t ws_bytes, void *stream);
