@@ -48,14 +48,21 @@
 // Work split (stream-K).  Blocks are numbered row-group-major (16-row group,
 // then tile) across all matrices of the call and dealt to all warps of the
 // grid in equal contiguous ranges, so every warp streams the same number of
-// bytes.  A warp keeps the accumulators of its current row group in
-// registers; a group it covers whole goes straight to y.  A group shared by
-// several warps is finished by the last of them to arrive: each contributor
-// writes its partial to the workspace and bumps the group's counter; the one
-// that completes the count adds the partials in warp order (so y is the same
-// on every call) and resets the counter to zero for the next call.  A warp
-// whose bounded wait gives up still arrives on every group it was to
-// contribute to, so the counters return to zero even then.
+// bytes (a CTA's warps hold consecutive ranges).  A warp keeps the
+// accumulators of its current row group in registers; a group it covers
+// whole goes straight to y.  A warp's first and last groups may be shared
+// with its neighbours: their sums wait in registers until the warp is done,
+// then go to its (by then free) ring in shared memory, and after a block
+// barrier the warp holding a shared group's first block in this CTA adds the
+// parts of the warps it spans, in warp order.  A group that stays inside the
+// CTA is then stored; one that crosses into another CTA is finished across
+// CTAs by the last CTA to arrive: each writes its part to the workspace and
+// bumps the group's counter, and the one that completes the count adds the
+// parts in CTA order (so y is the same on every call) and resets the counter
+// to zero for the next call.  Small matrices, where a 16-row group spans
+// many warps, so need no global fence or atomic for most groups.  A warp
+// whose bounded wait gives up still hands in (zero) parts, so every counter
+// sees all its arrivals and returns to zero even then.
 //
 // Launched with programmatic dependent launch: the weight copies and the
 // metadata loads start before the previous kernel in the stream has
@@ -105,7 +112,7 @@ struct __align__(64) Problem {
 struct __align__(64) Params {
     Problem prob[kMaxProblems];
     uint32_t *err;
-    float *part;    // workspace: [n_units][2][kSlotFloats] partials
+    float *part;    // workspace: [CTAs][2][kSlotFloats] partials of row groups shared by CTAs
     uint32_t *cnt;  // workspace: one arrival counter per row group (zero between calls)
     long long n_blocks;
     int n_problems, B;
@@ -200,9 +207,6 @@ __device__ __forceinline__ long long unit_start(long long u, long long n_blocks,
     return u * n_blocks / n_units;
 }
 
-__device__ __forceinline__ long long unit_of_block(long long b, long long n, int nu) {
-    return ((b + 1) * nu + n - 1) / n - 1;
-}
 
 // Start the copies of the stage at c into stage buffer st (completing on bar).
 __device__ __forceinline__ void issue(const Params &pr, const Cur &c, uint32_t st, uint32_t bar) {
@@ -404,43 +408,46 @@ __device__ __forceinline__ void store_y(const Problem &m, int B, const float (&a
 
 __device__ __forceinline__ int group_id(const Params &pr, int p, int grp) { return pr.prob[p].group0 + grp; }
 
-// The warp's accumulators of row group (p, grp) are complete for its part of
-// the group: store them, or hand them to the stream-K fix-up.  G0 is the
-// grouped index of the warp's first row group.
-__device__ __noinline__ void finish_group(const Params &pr, float4 a4, int p, int grp, int G0) {
-    const float acc[4] = {a4.x, a4.y, a4.z, a4.w};
-    const int lane = threadIdx.x & 31;
-    const int g = lane >> 2, q = lane & 3;
+// First block of CTA c's range (its warps' ranges in order).
+__device__ __forceinline__ long long cta_start(const Params &pr, long long c) {
+    return unit_start(c * kWarps, pr.n_blocks, pr.n_units);
+}
+
+// Row group (p, grp) holds blocks [gb0, gb1) of the grouped numbering.
+__device__ __forceinline__ void group_blocks(const Params &pr, int p, int grp, long long &gb0, long long &gb1) {
+    gb0 = pr.prob[p].block0 + static_cast<long long>(grp) * pr.prob[p].T;
+    gb1 = gb0 + pr.prob[p].T;
+}
+
+// The partial sums of a row group shared by several CTAs: this CTA's part
+// goes to the workspace (slot 0 for the CTA's first group, 1 for its last),
+// and the last CTA to arrive adds all parts in CTA order, stores y and
+// resets the group's counter.  Run by one warp.
+__device__ __noinline__ void cta_fixup(const Params &pr, float4 a4, int p, int grp) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
     const Problem &m = pr.prob[p];
-    const long long n = pr.n_blocks;
-    const long long u = static_cast<long long>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
-    const long long ub0 = unit_start(u, n, pr.n_units), ub1 = unit_start(u + 1, n, pr.n_units);
-    const long long gb0 = m.block0 + static_cast<long long>(grp) * m.T, gb1 = gb0 + m.T;
-    if (gb0 >= ub0 && gb1 <= ub1) {
-        store_y(m, pr.B, acc, grp, g, q);
-        return;
-    }
+    const int n_ctas = gridDim.x;
+    const long long c = blockIdx.x, c0 = cta_start(pr, c);
+    long long gb0, gb1;
+    group_blocks(pr, p, grp, gb0, gb1);
     const int G = m.group0 + grp;
-    const int slot = G == G0 ? 0 : 1;
-    float4 *mine = reinterpret_cast<float4 *>(pr.part + (static_cast<size_t>(u) * 2 + slot) * kSlotFloats) + lane;
+    float4 *mine = reinterpret_cast<float4 *>(pr.part + (static_cast<size_t>(c) * 2 + (gb0 <= c0 ? 0 : 1)) *
+                                                            kSlotFloats) + lane;
     __stcg(mine, a4);
     __threadfence();
     __syncwarp();
-    const long long uf = unit_of_block(gb0, n, pr.n_units), ul = unit_of_block(gb1 - 1, n, pr.n_units);
-    uint32_t n_contrib = 0;
-    for (long long v = uf; v <= ul; ++v)
-        if (unit_start(v, n, pr.n_units) < unit_start(v + 1, n, pr.n_units)) ++n_contrib;
+    // the CTAs whose ranges meet the group (a CTA's range is never empty)
+    long long cf = c, cl = c;
+    while (cf > 0 && cta_start(pr, cf) > gb0) --cf;
+    while (cl + 1 < n_ctas && cta_start(pr, cl + 1) < gb1) ++cl;
     uint32_t prev = 0;
     if (lane == 0) prev = atomicAdd(pr.cnt + G, 1u);
     prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
-    if (prev + 1 != n_contrib) return;
+    if (prev + 1 != static_cast<uint32_t>(cl - cf + 1)) return;
     __threadfence();
     float s[4] = {0.f, 0.f, 0.f, 0.f};
-    for (long long v = uf; v <= ul; ++v) {
-        const long long vs = unit_start(v, n, pr.n_units);
-        if (vs >= unit_start(v + 1, n, pr.n_units)) continue;
-        const Cur cv = locate(pr, vs, 0);
-        const int sl = group_id(pr, cv.p, cv.grp) == G ? 0 : 1;
+    for (long long v = cf; v <= cl; ++v) {
+        const int sl = gb0 <= cta_start(pr, v) ? 0 : 1;
         const float4 t =
             __ldcg(reinterpret_cast<const float4 *>(pr.part + (static_cast<size_t>(v) * 2 + sl) * kSlotFloats) + lane);
         s[0] += t.x;
@@ -452,8 +459,56 @@ __device__ __noinline__ void finish_group(const Params &pr, float4 a4, int p, in
     if (lane == 0) atomicExch(pr.cnt + G, 0u);
 }
 
+// After every warp of the CTA has put the sums of its split row groups in
+// its partial slots (slot 0: its first group, slot 1: its last; in its own
+// ring, which is free by then): each split group is completed by the warp
+// whose range holds the group's first block inside this CTA, adding the
+// parts of the warps it spans in warp order, then storing y or handing the
+// CTA's part to the fix-up across CTAs.
+__device__ __noinline__ void cta_combine(const Params &pr, uint32_t slots0) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+    const long long u = static_cast<long long>(blockIdx.x) * kWarps;
+    const long long c0 = unit_start(u, pr.n_blocks, pr.n_units), c1 = unit_start(u + kWarps, pr.n_blocks, pr.n_units);
+    const long long wb = unit_start(u + warp, pr.n_blocks, pr.n_units), we = unit_start(u + warp + 1, pr.n_blocks, pr.n_units);
+    if (wb >= we) return;
+    const Cur first = locate(pr, wb, 0), last = locate(pr, we - 1, 0);
+    for (int k = 0; k < 2; ++k) {
+        const Cur cg = k ? last : first;
+        if (k && cg.p == first.p && cg.grp == first.grp) break;
+        long long gb0, gb1;
+        group_blocks(pr, cg.p, cg.grp, gb0, gb1);
+        if (gb0 >= wb && gb1 <= we) continue;  // whole in this warp: stored already
+        if ((gb0 > c0 ? gb0 : c0) < wb) continue;  // an earlier warp completes it
+        float s[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int v = warp; v < kWarps; ++v) {
+            const long long vb = unit_start(u + v, pr.n_blocks, pr.n_units);
+            const long long ve = unit_start(u + v + 1, pr.n_blocks, pr.n_units);
+            if (vb >= gb1) break;
+            if (vb >= ve) continue;
+            const uint32_t sl = gb0 <= vb ? 0u : 1u;  // the group is warp v's first or last
+            const uint4 t = lds128(slots0 + static_cast<uint32_t>(v) * kStages * kStageBytes + sl * kGemvSlotBytes +
+                                   16u * lane);
+            s[0] += __uint_as_float(t.x);
+            s[1] += __uint_as_float(t.y);
+            s[2] += __uint_as_float(t.z);
+            s[3] += __uint_as_float(t.w);
+        }
+        if (gb0 >= c0 && gb1 <= c1)
+            store_y(pr.prob[cg.p], pr.B, s, cg.grp, g, q);
+        else
+            cta_fixup(pr, make_float4(s[0], s[1], s[2], s[3]), cg.p, cg.grp);
+    }
+}
+
 __device__ __forceinline__ float4 sum_halves(const float (&acc)[2][4]) {
     return make_float4(acc[0][0] + acc[1][0], acc[0][1] + acc[1][1], acc[0][2] + acc[1][2], acc[0][3] + acc[1][3]);
+}
+
+// Store the sums of a row group held whole by this warp.
+__device__ __forceinline__ void store_whole(const Params &pr, int p, int grp, const float (&acc)[2][4], int g,
+                                            int q) {
+    const float a[4] = {acc[0][0] + acc[1][0], acc[0][1] + acc[1][1], acc[0][2] + acc[1][2], acc[0][3] + acc[1][3]};
+    store_y(pr.prob[p], pr.B, a, grp, g, q);
 }
 
 // ---------------------------------------------------------------------------
@@ -469,14 +524,14 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
     const uint32_t bars = sb + static_cast<uint32_t>(warp) * kStages * 8u;
     const uint32_t ring = sb + kRingOff + static_cast<uint32_t>(warp) * kStages * kStageBytes;
     if (threadIdx.x == 0) grid_launch_dependents();
-    Cur cc;  // the stage being computed
-    {
-        const long long u = static_cast<long long>(blockIdx.x) * kWarps + warp;
-        const long long ub0 = unit_start(u, pr.n_blocks, pr.n_units);
-        const int nb = static_cast<int>(unit_start(u + 1, pr.n_blocks, pr.n_units) - ub0);
-        if (nb <= 0) return;
-        cc = locate(pr, ub0, nb);
-    }
+    const long long u = static_cast<long long>(blockIdx.x) * kWarps + warp;
+    const long long ub0 = unit_start(u, pr.n_blocks, pr.n_units);
+    const int nb = static_cast<int>(unit_start(u + 1, pr.n_blocks, pr.n_units) - ub0);
+    // The warp's range, then the row groups it shares with other warps
+    // completed together (a lambda, so that its early exits still reach the
+    // block barrier below).
+    auto body = [&]() {
+    Cur cc = locate(pr, ub0, nb);  // the stage being computed
 
     // The weights are never written by other kernels: start the copies and
     // the metadata loads before waiting for the previous grid.
@@ -513,6 +568,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
 
     int gp = cc.p, ggrp = cc.grp;  // the row group being accumulated
     const int G0 = group_id(pr, gp, ggrp);
+    // the sums of the warp's first row group when other warps share it
+    float4 first_part = make_float4(0.f, 0.f, 0.f, 0.f);
     grid_dependency_wait();  // x, y and the workspace may belong to earlier kernels
     const int gx = g < pr.B ? g : 0;  // batch rows past B repeat row 0; their outputs are dropped
     // The lane's shared-memory places (stage layout [row][tile][bytes]): raw
@@ -538,7 +595,14 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
             mn = load_meta<V>(pr.prob[cn.p], cn, lenn, g, tq, cn.j == 0);
         }
         if (cc.p != gp || cc.grp != ggrp) {
-            finish_group(pr, sum_halves(acc), gp, ggrp, G0);
+            // a group ends inside the range: the warp's whole group is stored,
+            // its first group (if another warp has part of it) is kept
+            long long gb0, gb1;
+            group_blocks(pr, gp, ggrp, gb0, gb1);
+            if (gb0 >= ub0)
+                store_whole(pr, gp, ggrp, acc, g, q);
+            else
+                first_part = sum_halves(acc);
 #pragma unroll
             for (int k = 0; k < 4; ++k) acc[0][k] = acc[1][k] = 0.f;
             gp = cc.p;
@@ -671,27 +735,41 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
         mc = mn;
         if (lenn > 0) advance(cn, lenn, pr);
     }
+    // the last group: whole in the range, or shared (its part goes to slot
+    // 0 when it is also the first group, else to slot 1)
+    long long gb0, gb1;
+    group_blocks(pr, gp, ggrp, gb0, gb1);
+    const long long ub1 = ub0 + nb;
+    float4 last_part = make_float4(0.f, 0.f, 0.f, 0.f);
     if (ok) {
-        finish_group(pr, sum_halves(acc), gp, ggrp, G0);
-        return;
+        if (gb0 >= ub0 && gb1 <= ub1)
+            store_whole(pr, gp, ggrp, acc, g, q);
+        else if (group_id(pr, gp, ggrp) == G0)
+            first_part = sum_halves(acc);
+        else
+            last_part = sum_halves(acc);
+    } else {
+        // A wait gave up (the error word says so; y is not valid): the
+        // shared groups get zero parts, so every counter still sees all its
+        // arrivals; the copies still in flight land first.
+        first_part = last_part = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (lane == 0)
+            for (int k = consumed; k < issued; ++k)
+                mbar_wait_s(bars + 8u * (k & 1), static_cast<uint32_t>(k >> 1) & 1u);
+        __syncwarp();
     }
-    // A wait gave up (the error word says so; y is not valid).  Still arrive
-    // on the current row group and every later one this warp shares, so each
-    // group's counter returns to zero, then let the copies still in flight
-    // land before the warp exits.
-    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int left = cc.left + cc.j;;) {
-        finish_group(pr, z, gp, ggrp, G0);
-        // blocks of this warp's range after the group just finished
-        left -= pr.prob[gp].T;
-        if (left <= 0) break;
-        if (++ggrp == pr.prob[gp].n_groups) {
-            ggrp = 0;
-            if (++gp == pr.n_problems) break;
-        }
-    }
-    if (lane == 0)
-        for (int k = consumed; k < issued; ++k) mbar_wait_s(bars + 8u * (k & 1), static_cast<uint32_t>(k >> 1) & 1u);
+    // the ring is free now: the two parts go to its first 1 KB
+    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(ring + 16u * lane), "f"(first_part.x),
+                 "f"(first_part.y), "f"(first_part.z), "f"(first_part.w)
+                 : "memory");
+    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(ring + kGemvSlotBytes + 16u * lane),
+                 "f"(last_part.x), "f"(last_part.y), "f"(last_part.z), "f"(last_part.w)
+                 : "memory");
+    };
+    if (nb > 0) body();
+    __syncthreads();
+    grid_dependency_wait();
+    cta_combine(pr, sb + kRingOff);
 }
 
 }  // namespace gemv
