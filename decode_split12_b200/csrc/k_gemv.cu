@@ -193,18 +193,28 @@ __device__ __forceinline__ void advance(Cur &c, int len, const Params &pr) {
     }
 }
 
-// Position of grouped block b (b < n_blocks), with `left` blocks to go.
+// Position of grouped block b (b < n_blocks), with `left` blocks to go.  (A
+// matrix has fewer than 2^32 / 2048 blocks, so 32-bit division serves.)
 __device__ __forceinline__ Cur locate(const Params &pr, long long b, int left) {
     int p = 0;
     while (p + 1 < pr.n_problems && pr.prob[p + 1].block0 <= b) ++p;
-    const long long local = b - pr.prob[p].block0;
-    const int T = pr.prob[p].T;
-    return Cur{p, static_cast<int>(local / T), static_cast<int>(local % T), left};
+    const uint32_t local = static_cast<uint32_t>(b - pr.prob[p].block0);
+    const uint32_t T = static_cast<uint32_t>(pr.prob[p].T);
+    const uint32_t grp = local / T;
+    return Cur{p, static_cast<int>(grp), static_cast<int>(local - grp * T), left};
 }
 
-// First block of warp unit u's range.
+// First block of warp unit u's range: floor(u * n_blocks / n_units), from a
+// double-precision quotient (the product is below 2^53) corrected to the
+// exact floor; cheaper than a 64-bit integer division.
 __device__ __forceinline__ long long unit_start(long long u, long long n_blocks, int n_units) {
-    return u * n_blocks / n_units;
+    const long long x = u * n_blocks;
+    long long q = static_cast<long long>(static_cast<double>(x) / static_cast<double>(n_units));
+    if (q * n_units > x)
+        --q;
+    else if ((q + 1) * n_units <= x)
+        ++q;
+    return q;
 }
 
 
@@ -468,8 +478,11 @@ __device__ __noinline__ void cta_fixup(const Params &pr, float4 a4, int p, int g
 __device__ __noinline__ void cta_combine(const Params &pr, uint32_t slots0) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
     const long long u = static_cast<long long>(blockIdx.x) * kWarps;
-    const long long c0 = unit_start(u, pr.n_blocks, pr.n_units), c1 = unit_start(u + kWarps, pr.n_blocks, pr.n_units);
-    const long long wb = unit_start(u + warp, pr.n_blocks, pr.n_units), we = unit_start(u + warp + 1, pr.n_blocks, pr.n_units);
+    // the CTA's warp boundaries, lane i holding the start of warp i's range
+    const long long bnd = unit_start(u + (lane <= kWarps ? lane : kWarps), pr.n_blocks, pr.n_units);
+    auto boundary = [&](int i) { return static_cast<long long>(__shfl_sync(0xFFFFFFFFu, bnd, i)); };
+    const long long c0 = boundary(0), c1 = boundary(kWarps);
+    const long long wb = boundary(warp), we = boundary(warp + 1);
     if (wb >= we) return;
     const Cur first = locate(pr, wb, 0), last = locate(pr, we - 1, 0);
     for (int k = 0; k < 2; ++k) {
@@ -481,8 +494,7 @@ __device__ __noinline__ void cta_combine(const Params &pr, uint32_t slots0) {
         if ((gb0 > c0 ? gb0 : c0) < wb) continue;  // an earlier warp completes it
         float s[4] = {0.f, 0.f, 0.f, 0.f};
         for (int v = warp; v < kWarps; ++v) {
-            const long long vb = unit_start(u + v, pr.n_blocks, pr.n_units);
-            const long long ve = unit_start(u + v + 1, pr.n_blocks, pr.n_units);
+            const long long vb = boundary(v), ve = boundary(v + 1);
             if (vb >= gb1) break;
             if (vb >= ve) continue;
             const uint32_t sl = gb0 <= vb ? 0u : 1u;  // the group is warp v's first or last
