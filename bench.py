@@ -795,10 +795,12 @@ def stack_extras(world, layers: int = 32, steps: int = 10):
     as one interleaved container), one pass = all layers; B = 1 and 8.
     Two forms: one grouped launch per layer over its six containers (pure
     weight streaming), and the activation chain, where the layer's down
-    output (BF16) is the next layer's input: per layer q, k, v, o in one
-    grouped launch (attention is outside the path: o reads the layer input
-    in its place), gate/up with the SwiGLU epilogue, down with a BF16
-    output.
+    output (BF16) feeds the next layer: per layer q, k, v, o in one grouped
+    launch (attention is outside the path: o reads the layer input in its
+    place), gate/up with the SwiGLU epilogue, down with a BF16 output, then
+    an RMS normalisation (torch, standing in for the model's norm layers,
+    which are outside the path) so the activations neither vanish nor blow
+    up over the layers.
     Plus an 8-expert MoE block (gate, up 14336x4096, down 4096x14336 per
     expert) with top-2 routing of 64 tokens: experts with >= 9 tokens use the
     skinny GEMM (rows padded to 16), the rest the GEMV."""
@@ -854,6 +856,7 @@ def stack_extras(world, layers: int = 32, steps: int = 10):
         h0 = dev16(wl.activations(B, Dm, B, 5000))
         hs = [h0] + [torch.empty((B, Dm), dtype=torch.int16, device="cuda") for _ in range(layers)]
         hid = torch.empty((B, F), dtype=torch.int16, device="cuda")
+        yd = torch.empty((B, Dm), dtype=torch.int16, device="cuda")
         yp = [torch.empty((B, shapes[n][0]), dtype=torch.float32, device="cuda") for n in ("q", "k", "v", "o")]
 
         def chain():
@@ -861,7 +864,9 @@ def stack_extras(world, layers: int = 32, steps: int = 10):
                 h = hs[l]
                 s12.s12_gemv_multi(lv[:4], [h] * 4, yp, ws=ws)
                 s12.s12_gemv_swiglu(lv[4], h, hid, ws=ws)
-                s12.s12_gemv_bf16(lv[5], hid, hs[l + 1], ws=ws)
+                s12.s12_gemv_bf16(lv[5], hid, yd, ws=ws)
+                hs[l + 1].view(torch.bfloat16).copy_(
+                    torch.nn.functional.rms_norm(yd.view(torch.bfloat16), (Dm,), eps=1e-6))
 
         g = capture(chain)
         for _ in range(3):
@@ -871,6 +876,7 @@ def stack_extras(world, layers: int = 32, steps: int = 10):
         out[f"chain_B{B}"] = {"ms_per_pass": round(t * 1e3, 3), "ms_per_token": round(t * 1e3 / B, 3),
                               "effective_bf16_GBs": round(2 * weights / t / 1e9, 1),
                               "hbm_frac": round(cbytes / t / 1e9 / hbm, 4), "launches_per_pass": 3 * layers,
+                              "norm": "torch rms_norm after each layer (outside the path), in the timed graph",
                               "output_finite": bool(torch.isfinite(last).all()),
                               "output_rms": float(last.pow(2).mean().sqrt())}
         del g
