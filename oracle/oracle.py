@@ -64,6 +64,12 @@ def _bind(lib: C.CDLL) -> C.CDLL:
     lib.oracle_encode_v2.restype = C.c_int
     lib.oracle_decode_v2.argtypes = [_P, _U64, _P]
     lib.oracle_decode_v2.restype = C.c_int
+    lib.oracle_container_bytes_v3.argtypes = [_U64, _U64, _U64]
+    lib.oracle_container_bytes_v3.restype = _I64
+    lib.oracle_encode_v3.argtypes = [_P, _U64, _U64, _P, _U64, _P]
+    lib.oracle_encode_v3.restype = C.c_int
+    lib.oracle_decode_v3.argtypes = [_P, _U64, _P]
+    lib.oracle_decode_v3.restype = C.c_int
     lib.oracle_silu_mul_f64.argtypes = [_P, _P, _I64, _P]
     lib.oracle_silu_mul_f64.restype = C.c_int
     lib.oracle_stats.argtypes = [_P, _U64, _P]
@@ -220,6 +226,31 @@ class Oracle:
         out = np.zeros((rows, cols), np.uint16)
         return int(self.lib.oracle_decode_v2(_ptr(blob), blob.size, _ptr(out)))
 
+    # -- container version 3 (packed 24-bit pairs) --
+    def container_bytes_v3(self, rows: int, cols: int, n_esc: int) -> int:
+        return int(self.lib.oracle_container_bytes_v3(rows, cols, n_esc))
+
+    def encode_v3(self, w: np.ndarray) -> np.ndarray:
+        w = np.ascontiguousarray(w, dtype=np.uint16)
+        rows, cols = w.shape
+        nbytes = C.c_uint64(0)
+        _check(self.lib.oracle_encode_v3(_ptr(w), rows, cols, None, 0, C.byref(nbytes)), "encode_v3 size")
+        out = np.zeros(nbytes.value, np.uint8)
+        _check(self.lib.oracle_encode_v3(_ptr(w), rows, cols, _ptr(out), out.size, C.byref(nbytes)), "encode_v3")
+        return out
+
+    def decode_v3(self, blob: np.ndarray) -> np.ndarray:
+        blob = np.ascontiguousarray(blob, dtype=np.uint8)
+        rows, cols = self.shape_of(blob)
+        out = np.zeros((rows, cols), np.uint16)
+        _check(self.lib.oracle_decode_v3(_ptr(blob), blob.size, _ptr(out)), "decode_v3")
+        return out
+
+    def decode_v3_rc(self, blob: np.ndarray) -> int:
+        blob = np.ascontiguousarray(blob, dtype=np.uint8)
+        rows, cols = self.shape_of(blob)
+        out = np.zeros((rows, cols), np.uint16)
+        return int(self.lib.oracle_decode_v3(_ptr(blob), blob.size, _ptr(out)))
     def silu_mul_f64(self, g: np.ndarray, u: np.ndarray) -> np.ndarray:
         """h = silu(g) * u elementwise (the C oracle's gated-MLP activation)."""
         g = np.ascontiguousarray(g, dtype=np.float64)

@@ -97,6 +97,7 @@ static uint16_t get_u16(const uint8_t *p) {
     return (uint16_t)(p[0] | (p[1] << 8));
 }
 
+
 static uint64_t pad_to_align(uint64_t n) {
     return (n + ORACLE_ALIGN - 1) / ORACLE_ALIGN * ORACLE_ALIGN;
 }
@@ -475,6 +476,134 @@ int oracle_decode_v2(const uint8_t *blob, uint64_t bytes, uint16_t *out) {
                 }
             }
             if (seen != count) return ORACLE_ERR_CORRUPT;
+        }
+        if (k != hi) return ORACLE_ERR_CORRUPT;
+    }
+    return ORACLE_OK;
+}
+
+/* ---------------------------------------------------------------------- */
+/* Container version 3: packed 24-bit pairs.  [T] technical deep dive says
+ * the 12-bit representation is packed into 3-byte words, two weights per
+ * word.  Reading (the plainest one with this build's 12-bit split): weights
+ * 2i and 2i+1 (row-major, always in the same tile) form pair i, stored as
+ * three consecutive bytes
+ *     byte 3i     raw(w[2i])
+ *     byte 3i+1   raw(w[2i+1])
+ *     byte 3i+2   code(w[2i]) | code(w[2i+1]) << 4
+ * in one pair plane u8[rows*cols*3/2] that takes the place of the raw and
+ * code planes.  Base choice, codes, escapes, the base and esc_off planes and
+ * the header (version = 3) are those of version 1; every plane starts on a
+ * 256-byte boundary. */
+typedef struct {
+    uint64_t rows, cols, n_tiles, n_esc;
+    uint64_t off_pair, off_base, off_esc_off, off_esc, total;
+} oracle_layout3;
+
+static int layout3_for(uint64_t rows, uint64_t cols, uint64_t n_esc, oracle_layout3 *L) {
+    if (cols == 0 || cols % ORACLE_TILE != 0 || rows == 0) return ORACLE_ERR_SHAPE;
+    if (rows > (UINT64_C(1) << 40) / cols) return ORACLE_ERR_SHAPE;
+    L->rows = rows;
+    L->cols = cols;
+    L->n_tiles = rows * (cols / ORACLE_TILE);
+    L->n_esc = n_esc;
+    L->off_pair = pad_to_align(ORACLE_HEADER_USED);
+    L->off_base = L->off_pair + pad_to_align(rows * cols / 2 * 3);
+    L->off_esc_off = L->off_base + pad_to_align(L->n_tiles);
+    L->off_esc = L->off_esc_off + pad_to_align(4 * (L->n_tiles + 1));
+    L->total = L->off_esc + pad_to_align(2 * L->n_esc);
+    return ORACLE_OK;
+}
+
+int64_t oracle_container_bytes_v3(uint64_t rows, uint64_t cols, uint64_t n_esc) {
+    oracle_layout3 L;
+    int rc = layout3_for(rows, cols, n_esc, &L);
+    if (rc != ORACLE_OK) return rc;
+    return (int64_t)L.total;
+}
+
+/* Encoder, version 3. */
+int oracle_encode_v3(const uint16_t *w, uint64_t rows, uint64_t cols, uint8_t *dst, uint64_t cap,
+                     uint64_t *bytes_out) {
+    if (!w || !bytes_out) return ORACLE_ERR_ARG;
+    oracle_layout3 L;
+    int rc = layout3_for(rows, cols, 0, &L);
+    if (rc != ORACLE_OK) return rc;
+    uint64_t n_esc = 0;
+    for (uint64_t t = 0; t < L.n_tiles; t++) {
+        uint32_t b;
+        n_esc += (uint64_t)oracle_tile_base(w + t * ORACLE_TILE, &b, NULL);
+    }
+    if (n_esc > 0xFFFFFFFFull) return ORACLE_ERR_SHAPE; /* esc_off is u32 */
+    layout3_for(rows, cols, n_esc, &L);
+    *bytes_out = L.total;
+    if (!dst) return ORACLE_OK;
+    if (cap < L.total) return ORACLE_ERR_CAPACITY;
+
+    memset(dst, 0, L.total);
+    memcpy(dst, "S12\0", 4);
+    put_u32(dst + 4, 3);
+    put_u64(dst + 8, rows);
+    put_u64(dst + 16, cols);
+    put_u32(dst + 24, ORACLE_TILE);
+    put_u32(dst + 28, 0);
+    put_u64(dst + 32, n_esc);
+    uint8_t *pair = dst + L.off_pair, *base = dst + L.off_base, *off = dst + L.off_esc_off, *esc = dst + L.off_esc;
+    uint64_t written = 0;
+    for (uint64_t t = 0; t < L.n_tiles; t++) {
+        const uint16_t *tw = w + t * ORACLE_TILE;
+        uint32_t b;
+        oracle_tile_base(tw, &b, NULL);
+        base[t] = (uint8_t)b;
+        put_u32(off + 4 * t, (uint32_t)written);
+        /* the tile's raw bytes and codes as version 1 lays them out, then
+         * regrouped into 3-byte pairs */
+        uint8_t raw_t[ORACLE_TILE], code_t[ORACLE_TILE / 2];
+        pack_tile(tw, b, 0, raw_t, code_t, esc, &written);
+        uint8_t *pt = pair + 3 * (t * ORACLE_TILE / 2);
+        for (uint32_t i = 0; i < ORACLE_TILE / 2; i++) {
+            pt[3 * i] = raw_t[2 * i];
+            pt[3 * i + 1] = raw_t[2 * i + 1];
+            pt[3 * i + 2] = code_t[i];
+        }
+    }
+    put_u32(off + 4 * L.n_tiles, (uint32_t)written);
+    return ORACLE_OK;
+}
+
+/* Decoder, version 3, with the checks of version 1: offsets start at 0,
+ * end at n_esc and never decrease; each tile's code-15 count equals its
+ * offset span; bases are at most 241. */
+int oracle_decode_v3(const uint8_t *blob, uint64_t bytes, uint16_t *out) {
+    if (!blob || !out) return ORACLE_ERR_ARG;
+    if (bytes < ORACLE_HEADER_USED || memcmp(blob, "S12\0", 4) != 0) return ORACLE_ERR_CORRUPT;
+    if (get_u32(blob + 4) != 3 || get_u32(blob + 24) != ORACLE_TILE || get_u32(blob + 28) != 0)
+        return ORACLE_ERR_CORRUPT;
+    for (int i = 40; i < 64; i++)
+        if (blob[i] != 0) return ORACLE_ERR_CORRUPT;
+    uint64_t rows = get_u64(blob + 8), cols = get_u64(blob + 16), n_esc = get_u64(blob + 32);
+    oracle_layout3 L;
+    if (layout3_for(rows, cols, n_esc, &L) != ORACLE_OK) return ORACLE_ERR_CORRUPT;
+    if (n_esc > rows * cols || bytes < L.total) return ORACLE_ERR_CORRUPT;
+    const uint8_t *pair = blob + L.off_pair, *base = blob + L.off_base, *off = blob + L.off_esc_off;
+    const uint8_t *esc = blob + L.off_esc;
+    if (get_u32(off) != 0 || get_u32(off + 4 * L.n_tiles) != n_esc) return ORACLE_ERR_CORRUPT;
+    for (uint64_t t = 0; t < L.n_tiles; t++) {
+        const uint64_t lo = get_u32(off + 4 * t), hi = get_u32(off + 4 * (t + 1));
+        const uint32_t b = base[t];
+        if (hi < lo || hi > n_esc || b > ORACLE_MAX_BASE) return ORACLE_ERR_CORRUPT;
+        uint64_t k = lo;
+        for (uint32_t i = 0; i < ORACLE_TILE; i++) {
+            const uint64_t pos = t * ORACLE_TILE + i, p = pos / 2;
+            const uint8_t rb = pair[3 * p + (pos % 2)];
+            const uint32_t c = (pos % 2 == 0) ? (pair[3 * p + 2] & 0x0Fu) : (uint32_t)(pair[3 * p + 2] >> 4);
+            if (c < ORACLE_ESCAPE_CODE) {
+                out[pos] = (uint16_t)(((uint32_t)(rb & 0x80) << 8) | ((b + c) << 7) | (rb & 0x7Fu));
+            } else {
+                if (k >= hi) return ORACLE_ERR_CORRUPT;
+                out[pos] = get_u16(esc + 2 * k);
+                k++;
+            }
         }
         if (k != hi) return ORACLE_ERR_CORRUPT;
     }

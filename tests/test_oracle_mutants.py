@@ -56,6 +56,15 @@ MUTANTS = {
          "        tmeta[2 * t + 1] = (uint8_t)b;\n        tmeta[2 * t] = (uint8_t)count;"),
         ("uint32_t b = tmeta[2 * t], count = tmeta[2 * t + 1], seen = 0;",
          "uint32_t b = tmeta[2 * t + 1], count = tmeta[2 * t], seen = 0;")],
+    "v3_pair_raw_bytes_swapped": [("            pt[3 * i] = raw_t[2 * i];\n            pt[3 * i + 1] = raw_t[2 * i + 1];",
+                                   "            pt[3 * i] = raw_t[2 * i + 1];\n            pt[3 * i + 1] = raw_t[2 * i];")],
+    "v3_pair_nibbles_swapped_consistently": [
+        ("            pt[3 * i + 2] = code_t[i];",
+         "            pt[3 * i + 2] = (uint8_t)((code_t[i] >> 4) | (code_t[i] << 4));"),
+        ("(pos % 2 == 0) ? (pair[3 * p + 2] & 0x0Fu) : (uint32_t)(pair[3 * p + 2] >> 4)",
+         "(pos % 2 == 1) ? (pair[3 * p + 2] & 0x0Fu) : (uint32_t)(pair[3 * p + 2] >> 4)")],
+    "v3_pair_plane_unpadded": [("L->off_base = L->off_pair + pad_to_align(rows * cols / 2 * 3);",
+                                "L->off_base = L->off_pair + rows * cols / 2 * 3;")],
     "escape_stored_byte_swapped": [("esc[2 * *written] = (uint8_t)(v & 0xFF);\n            esc[2 * *written + 1] = (uint8_t)(v >> 8);",
                                     "esc[2 * *written] = (uint8_t)(v >> 8);\n            esc[2 * *written + 1] = (uint8_t)(v & 0xFF);")],
 }
@@ -112,6 +121,21 @@ def _battery(o: Oracle):
     bad = b2.copy()
     bad[off_t + 2 * k + 1] += 1
     assert o.decode_v2_rc(bad) != 0
+    # container version 3: the hand-derived golden, round trip, agreement
+    # with version 1's planes
+    g3 = load_golden("two_tiles_v3.json")
+    e3 = golden_expected_bytes(d)
+    for lo, hi in g3["clear"]:
+        e3[lo:hi] = 0
+    for item in g3["patch"]:
+        chunk = np.frombuffer(bytes.fromhex(item[1]) * (item[2] if len(item) > 2 else 1), np.uint8)
+        e3[item[0]:item[0] + chunk.size] = chunk
+    assert np.array_equal(o.encode_v3(w), e3)
+    assert np.array_equal(o.decode_v3(o.encode_v3(wv)), wv)
+    b3 = o.encode_v3(w2)
+    pr = b3[256:256 + 16 * 1024 * 3 // 2].reshape(-1, 3)
+    assert np.array_equal(pr[:, 2], b1[256 + 16 * 1024:256 + 16 * 1024 + 8192])
+    assert np.array_equal(pr[:, 0], b1[256:256 + 16 * 1024:2])
     # gated-MLP activation: textbook values of t * logistic(t)
     e = np.e
     h = o.silu_mul_f64(np.array([1.0, 2.0, 64.0, -64.0, 0.0]), np.array([2.0, 1.0, 3.0, 3.0, 5.0]))
