@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Para
             const int nt = static_cast<int>(min(static_cast<long long>(kChunkTiles), p.n_tiles - t0));
             mb = mo = me = 0;
             if (lane < nt) {
-                if (V == 1) {
+                if (V != 2) {
                     mb = __ldg(static_cast<const uint8_t *>(p.meta) + t);
                     mo = __ldg(p.off + t);
                 } else {
@@ -148,7 +148,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Para
                     mo = w >> 8;
                 }
             }
-            if (V == 1 && lane == 31) me = __ldg(p.off + t0 + nt);
+            if (V != 2 && lane == 31) me = __ldg(p.off + t0 + nt);
         };
         // version 2: escapes before the first tile of the range
         uint32_t carry = 0;
@@ -192,7 +192,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Para
             if (c + kAhead < c1) load(c + kAhead, rb[kAhead - 1], ro[kAhead - 1], re[kAhead - 1]);
             // first escape of each tile, and the chunk's span [e0, e1)
             uint32_t first, e1;
-            if (V == 1) {
+            if (V != 2) {
                 first = mo;
                 e1 = __shfl_sync(0xFFFFFFFFu, me, 31);
             } else {
@@ -225,8 +225,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Para
             if (lane == 0) {
                 const uint32_t esc_bytes = n_stage ? a1 - a0 : 0u;
                 bar_expect_tx(full + 8 * s, nt * 192u + esc_bytes);
-                bulk_load(st, p.raw + t0 * 128, nt * 128u, full + 8 * s);
-                bulk_load(st + kRawB, p.code + t0 * 64, nt * 64u, full + 8 * s);
+                if (V == 3) {
+                    // the pair plane: a tile's raw bytes and codes, 192 bytes
+                    bulk_load(st, p.raw + t0 * 192, nt * 192u, full + 8 * s);
+                } else {
+                    bulk_load(st, p.raw + t0 * 128, nt * 128u, full + 8 * s);
+                    bulk_load(st + kRawB, p.code + t0 * 64, nt * 64u, full + 8 * s);
+                }
                 if (esc_bytes)
                     bulk_load(st + kOffEsc, reinterpret_cast<const uint8_t *>(p.esc) + a0, esc_bytes, full + 8 * s);
             }
@@ -263,12 +268,30 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Para
             uint2 code = make_uint2(0, 0);
             uint32_t base = 0, lo = 0, hi = 0;
             if (active) {
-                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                             : "=r"(raw.x), "=r"(raw.y), "=r"(raw.z), "=r"(raw.w)
-                             : "r"(st + tl * 128 + piece * 16));
-                asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
-                             : "=r"(code.x), "=r"(code.y)
-                             : "r"(st + kRawB + tl * 64 + piece * 8));
+                if (V == 3) {
+                    // 8 pairs of 3 bytes: raw, raw, two codes; regrouped
+                    // into the 16 raw bytes and 8 code bytes of version 1
+                    uint32_t q[6];
+                    const uint32_t a = st + tl * 192 + piece * 24;
+#pragma unroll
+                    for (int h = 0; h < 3; ++h)
+                        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
+                                     : "=r"(q[2 * h]), "=r"(q[2 * h + 1])
+                                     : "r"(a + 8 * h));
+                    raw.x = prmt(q[0], q[1], 0x4310u);  // bytes 0 1 3 4
+                    raw.y = prmt(q[1], q[2], 0x6532u);  // bytes 6 7 9 10
+                    raw.z = prmt(q[3], q[4], 0x4310u);  // bytes 12 13 15 16
+                    raw.w = prmt(q[4], q[5], 0x6532u);  // bytes 18 19 21 22
+                    code.x = prmt(prmt(q[0], q[1], 0x0052u), q[2], 0x7410u);  // bytes 2 5 8 11
+                    code.y = prmt(prmt(q[3], q[4], 0x0052u), q[5], 0x7410u);  // bytes 14 17 20 23
+                } else {
+                    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(raw.x), "=r"(raw.y), "=r"(raw.z), "=r"(raw.w)
+                                 : "r"(st + tl * 128 + piece * 16));
+                    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
+                                 : "=r"(code.x), "=r"(code.y)
+                                 : "r"(st + kRawB + tl * 64 + piece * 8));
+                }
                 base = lds32(meta + 4 * tl);
                 lo = lds32(meta + 4 * (kChunkTiles + 1) + 4 * tl);
                 // the tile's span ends where the next one starts (the chunk's
@@ -364,8 +387,8 @@ int run_decode(const s12_view *v, uint16_t *out, unsigned long long *hist, uint3
     dec::Params p;
     p.raw = v->raw;
     p.code = v->code;
-    p.meta = V == 1 ? static_cast<const void *>(v->base) : static_cast<const void *>(v->tmeta);
-    p.off = V == 1 ? v->esc_off : v->row_esc;
+    p.meta = V != 2 ? static_cast<const void *>(v->base) : static_cast<const void *>(v->tmeta);
+    p.off = V != 2 ? v->esc_off : v->row_esc;
     p.esc = v->esc;
     p.n_esc = static_cast<uint32_t>(v->n_esc);
     p.n_tiles = static_cast<long long>(v->n_tiles);
@@ -389,12 +412,14 @@ int run_decode(const s12_view *v, uint16_t *out, unsigned long long *hist, uint3
 }  // namespace
 
 int launch_decode(const s12_view *v, uint16_t *out, uint32_t *err, cudaStream_t stream) {
+    if (v->version == 3) return run_decode<3, false>(v, out, nullptr, err, stream);
     return v->version == 1 ? run_decode<1, false>(v, out, nullptr, err, stream)
                            : run_decode<2, false>(v, out, nullptr, err, stream);
 }
 
 int launch_stats_hist(const s12_view *v, unsigned long long *hist, cudaStream_t stream) {
     if (cudaMemsetAsync(hist, 0, 256 * sizeof(unsigned long long), stream) != cudaSuccess) return S12_ERR_CUDA;
+    if (v->version == 3) return run_decode<3, true>(v, nullptr, hist, nullptr, stream);
     return v->version == 1 ? run_decode<1, true>(v, nullptr, hist, nullptr, stream)
                            : run_decode<2, true>(v, nullptr, hist, nullptr, stream);
 }

@@ -22,11 +22,13 @@ bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3) == 0;
 }  // namespace
 
 int check_view(const s12_view *v) {
-    if (!v || !v->container || !v->raw || !v->code || !v->esc) return S12_ERR_ARG;
+    if (!v || !v->container || !v->raw || !v->esc) return S12_ERR_ARG;
     if (v->version == 1) {
-        if (!v->base || !v->esc_off) return S12_ERR_ARG;
+        if (!v->code || !v->base || !v->esc_off) return S12_ERR_ARG;
     } else if (v->version == 2) {
-        if (!v->tmeta || !v->row_esc) return S12_ERR_ARG;
+        if (!v->code || !v->tmeta || !v->row_esc) return S12_ERR_ARG;
+    } else if (v->version == 3) {
+        if (!v->base || !v->esc_off) return S12_ERR_ARG;  // raw = the pair plane, no code plane
     } else {
         return S12_ERR_ARG;
     }
@@ -193,7 +195,7 @@ int s12_open(const void *container, size_t bytes, s12_view *out) {
     if (cudaMemcpy(h, container, sizeof h, cudaMemcpyDeviceToHost) != cudaSuccess) return S12_ERR_CUDA;
     if (std::memcmp(h, "S12\0", 4) != 0) return S12_ERR_CORRUPT;
     const uint32_t version = get_u32(h + 4);
-    if ((version != 1 && version != 2) || get_u32(h + 24) != static_cast<uint32_t>(kTile) || get_u32(h + 28) != 0)
+    if (version < 1 || version > 3 || get_u32(h + 24) != static_cast<uint32_t>(kTile) || get_u32(h + 28) != 0)
         return S12_ERR_CORRUPT;
     for (int i = 40; i < 64; ++i)
         if (h[i]) return S12_ERR_CORRUPT;
@@ -216,6 +218,15 @@ int s12_open(const void *container, size_t bytes, s12_view *out) {
         out->container_bytes = g.total;
         out->raw = c + g.off_raw;
         out->code = c + g.off_code;
+        out->base = c + g.off_base;
+        out->esc_off = reinterpret_cast<const uint32_t *>(c + g.off_esc_off);
+        out->esc = reinterpret_cast<const uint16_t *>(c + g.off_esc);
+    } else if (version == 3) {
+        const Geometry3 g = geometry3(rows, cols, n_esc);
+        if (g.total > bytes) return S12_ERR_CORRUPT;
+        out->n_tiles = g.n_tiles;
+        out->container_bytes = g.total;
+        out->raw = c + g.off_pair;  // the pair plane; code stays NULL
         out->base = c + g.off_base;
         out->esc_off = reinterpret_cast<const uint32_t *>(c + g.off_esc_off);
         out->esc = reinterpret_cast<const uint16_t *>(c + g.off_esc);
@@ -263,7 +274,7 @@ int gemv_check(const s12_view *views, int count, const uint16_t *const *x, int B
         if (rc != S12_OK) return rc;
         if (!x[i] || !y[i]) return S12_ERR_ARG;
         if (views[i].rows > 0x7FFFFFFFull || views[i].cols > 0x7FFFFFFFull) return S12_ERR_SHAPE;
-        if (views[i].version != views[0].version) return S12_ERR_ARG;
+        if (views[i].version != views[0].version || views[i].version > 2) return S12_ERR_ARG;
         const int o = out ? out[i] : kGemvOutF32;
         if (o != kGemvOutF32 && o != kGemvOutSwiglu && o != kGemvOutBf16) return S12_ERR_ARG;
         if (o == kGemvOutSwiglu && views[i].rows % 16 != 0) return S12_ERR_SHAPE;
@@ -418,7 +429,7 @@ int s12_stats(const s12_view *v, s12_stats_t *out, void *ws, size_t ws_bytes, vo
     out->n_esc = v->n_esc;
     out->container_bytes = v->container_bytes;
     out->payload_bytes = nw + nw / 2;
-    out->header_bytes = v->version == 1 ? v->n_tiles * 5 : v->n_tiles * 2 + 4 * (v->rows + 1);
+    out->header_bytes = v->version == 2 ? v->n_tiles * 2 + 4 * (v->rows + 1) : v->n_tiles * 5;
     out->escape_bytes = 2 * v->n_esc;
     out->escape_rate = static_cast<double>(v->n_esc) / static_cast<double>(nw);
     out->bits_per_weight = 8.0 * static_cast<double>(v->container_bytes) / static_cast<double>(nw);

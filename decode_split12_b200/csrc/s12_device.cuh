@@ -70,6 +70,28 @@ __host__ __device__ inline Geometry2 geometry2(uint64_t rows, uint64_t cols, uin
     return g;
 }
 
+// Plane offsets of a version 3 container (packed 24-bit pairs): weights 2i
+// and 2i+1 stored as raw(2i), raw(2i+1), code(2i) | code(2i+1) << 4 in one
+// pair plane, then the base, offset and escape planes of version 1.
+struct Geometry3 {
+    uint64_t rows, cols, n_tiles, n_esc;
+    uint64_t off_pair, off_base, off_esc_off, off_esc, total;
+};
+
+__host__ __device__ inline Geometry3 geometry3(uint64_t rows, uint64_t cols, uint64_t n_esc) {
+    Geometry3 g;
+    g.rows = rows;
+    g.cols = cols;
+    g.n_tiles = rows * (cols / kTile);
+    g.n_esc = n_esc;
+    g.off_pair = kHeaderBytes;
+    g.off_base = g.off_pair + align_up(rows * cols / 2 * 3, kAlign);
+    g.off_esc_off = g.off_base + align_up(g.n_tiles, kAlign);
+    g.off_esc = g.off_esc_off + align_up(4 * (g.n_tiles + 1), kAlign);
+    g.total = g.off_esc + align_up(2 * n_esc, kAlign);
+    return g;
+}
+
 // ---------------------------------------------------------------------------
 // Bounded waiting.  Every spin in these kernels gives up after about a second
 // at full clock, sets S12_FLAG_TIMEOUT and lets the caller unwind.

@@ -95,7 +95,13 @@ extern "C" {
  * pointers into the caller's container buffer.  A version 1 container has
  * `base` and `esc_off` (and NULL tmeta/row_esc); a version 2 container (the
  * compact tile header of s12_to_v2_host) has `tmeta` and `row_esc` (and NULL
- * base/esc_off).  Every kernel call reads either version. */
+ * base/esc_off).  A version 3 container (packed 24-bit pairs, [T] technical
+ * deep dive: weights 2i and 2i+1 stored as raw(2i), raw(2i+1),
+ * code(2i) | code(2i+1) << 4 in one pair plane of rows*cols*3/2 bytes, then
+ * version 1's base, esc_off and esc planes) has `raw` pointing at the pair
+ * plane, NULL `code`, and `base`/`esc_off` as version 1.  Decode and stats
+ * read all three versions; the fused GEMV and GEMM read versions 1 and 2
+ * (S12_ERR_ARG for version 3). */
 typedef struct s12_view {
     uint64_t rows;            /* output features (N)                      */
     uint64_t cols;            /* input features (K), multiple of 128      */
@@ -103,12 +109,12 @@ typedef struct s12_view {
     uint64_t n_esc;           /* escaped weights                          */
     uint64_t container_bytes; /* total size, multiple of 256              */
     const void *container;    /* start of the container                   */
-    const uint8_t *raw;       /* u8 [rows*cols]                           */
-    const uint8_t *code;      /* u8 [rows*cols/2]                         */
+    const uint8_t *raw;       /* u8 [rows*cols] (v3: pairs, rows*cols*3/2) */
+    const uint8_t *code;      /* u8 [rows*cols/2] (v3: NULL)              */
     const uint8_t *base;      /* version 1: u8 [n_tiles]                  */
     const uint32_t *esc_off;  /* version 1: u32[n_tiles+1]                */
     const uint16_t *esc;      /* u16[n_esc]                               */
-    uint32_t version;         /* 1 or 2                                   */
+    uint32_t version;         /* 1, 2 or 3                                */
     uint32_t reserved;        /* 0                                        */
     const uint16_t *tmeta;    /* version 2: u16[n_tiles], base | count<<8 */
     const uint32_t *row_esc;  /* version 2: u32[rows+1], escapes before r */
@@ -118,7 +124,7 @@ typedef struct s12_stats_t {
     uint64_t rows, cols, n_tiles, n_esc;
     uint64_t container_bytes; /* everything, padding included            */
     uint64_t payload_bytes;   /* raw + code = 1.5 bytes per weight       */
-    uint64_t header_bytes;    /* v1: 5 per tile; v2: 2 per tile + 4 per row */
+    uint64_t header_bytes;    /* v1, v3: 5 per tile; v2: 2 per tile + 4 per row */
     uint64_t escape_bytes;    /* 2 bytes per escape                      */
     double escape_rate;       /* n_esc / (rows*cols)                     */
     double bits_per_weight;   /* 8 * container_bytes / (rows*cols)       */
@@ -171,7 +177,7 @@ int s12_encode(const uint16_t *w, int64_t rows, int64_t cols, void *dst, size_t 
 /* Follows: the container layout above, which restates [M] section 1 (the
  * BF16 bit fields) and [T] key points (tile base, escape stream).
  * Validate the 64-byte header of a container (device, `bytes` long, version
- * 1 or 2) and fill *out with its shape, version and plane pointers.  Copies
+ * 1, 2 or 3) and fill *out with its shape, version and plane pointers.  Copies
  * the header to the host and so SYNCHRONISES (the legacy default stream).
  * S12_ERR_CORRUPT on a bad magic, version, tile size, flags, shape or a size
  * above `bytes`. */

@@ -264,3 +264,57 @@ def test_v2_stats_match_v1(s12, oracle):
     assert st["exp_entropy_bits"] == pytest.approx(ref["exp_entropy_bits"], abs=1e-12)
     assert st["header_bytes"] == 2 * view.n_tiles + 4 * (view.rows + 1)
     assert st["n_esc"] == ref["n_esc"]
+
+
+# ---------------------------------------------------------------------------
+# container version 3 (packed 24-bit pairs), built by the oracle
+
+@pytest.mark.parametrize("order", ["natural", "shuffled"])
+def test_v3_decode_all_patterns(s12, oracle, order):
+    """All 65,536 BF16 patterns as a version 3 container (two weights per
+    3 bytes; [T] technical deep dive): the GPU decode gives every bit back."""
+    w = _all_patterns(order)
+    view = s12.s12_open(blob_to_dev(oracle.encode_v3(w)))
+    assert view.version == 3
+    flag = new_flag()
+    out = s12.s12_decode(view, err_flag=flag)
+    torch.cuda.synchronize()
+    assert np.array_equal(from_dev_u16(out), w)
+    assert int(flag.item()) == 0
+
+
+@pytest.mark.parametrize("shape", [(1, 128), (3, 384), (67, 384), (300, 1152), (5, 14336)])
+@pytest.mark.parametrize("rate", [0.0003, 0.10])
+def test_v3_decode_shapes_and_escape_rates(s12, oracle, shape, rate):
+    r, c = shape
+    w, _ = wl.escape_stress(rate, 3 * r + c, r, c)
+    view = s12.s12_open(blob_to_dev(oracle.encode_v3(w)))
+    flag = new_flag()
+    out = s12.s12_decode(view, err_flag=flag)
+    torch.cuda.synchronize()
+    assert np.array_equal(from_dev_u16(out), w)
+    assert int(flag.item()) == 0
+
+
+def test_v3_decode_full_size_and_stats(s12, oracle):
+    """8192 x 8192 at 2 % escapes as a version 3 container: bit-exact; its
+    statistics equal the oracle's of the version 1 container; the fused
+    products refuse version 3 (they read versions 1 and 2)."""
+    w, planted = wl.escape_stress(0.02, seed=1)
+    view = s12.s12_open(blob_to_dev(oracle.encode_v3(w)))
+    assert view.n_esc == planted
+    flag = new_flag()
+    out = s12.s12_decode(view, err_flag=flag)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), to_dev(w))
+    assert int(flag.item()) == 0
+    small = wl.student_t_scaled(300, 1152, 6)
+    ref = oracle.stats(oracle.encode(small))
+    v3 = s12.s12_open(blob_to_dev(oracle.encode_v3(small)))
+    st = s12.s12_stats(v3)
+    assert st["exp_hist"] == [int(h) for h in ref["exp_hist"]]
+    assert st["n_esc"] == ref["n_esc"]
+    with pytest.raises(s12.S12Error):
+        s12.s12_gemv(v3, to_dev(wl.activations(1, 1152, 0)))
+    with pytest.raises(s12.S12Error):
+        s12.s12_gemm_skinny(v3, to_dev(wl.activations(16, 1152, 0)))
