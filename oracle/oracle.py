@@ -70,6 +70,14 @@ def _bind(lib: C.CDLL) -> C.CDLL:
     lib.oracle_encode_v3.restype = C.c_int
     lib.oracle_decode_v3.argtypes = [_P, _U64, _P]
     lib.oracle_decode_v3.restype = C.c_int
+    lib.oracle_container_bytes_v4.argtypes = [_U64, _U64, _U64]
+    lib.oracle_container_bytes_v4.restype = _I64
+    lib.oracle_encode_v4.argtypes = [_P, _U64, _U64, _P, _U64, _P]
+    lib.oracle_encode_v4.restype = C.c_int
+    lib.oracle_decode_v4.argtypes = [_P, _U64, _P]
+    lib.oracle_decode_v4.restype = C.c_int
+    lib.oracle_symbol_table.argtypes = [_P, _U64, _P]
+    lib.oracle_symbol_table.restype = _U64
     lib.oracle_silu_mul_f64.argtypes = [_P, _P, _I64, _P]
     lib.oracle_silu_mul_f64.restype = C.c_int
     lib.oracle_stats.argtypes = [_P, _U64, _P]
@@ -259,6 +267,39 @@ class Oracle:
         h = np.zeros_like(g)
         _check(self.lib.oracle_silu_mul_f64(_ptr(g), _ptr(u), g.size, _ptr(h)), "silu_mul")
         return h
+
+    # -- container version 4 (sign-and-exponent symbol codes) --
+    def container_bytes_v4(self, rows: int, cols: int, n_esc: int) -> int:
+        return int(self.lib.oracle_container_bytes_v4(rows, cols, n_esc))
+
+    def symbol_table(self, w: np.ndarray):
+        """(table of 32 u16, number of weights outside it)."""
+        w = np.ascontiguousarray(w, dtype=np.uint16).reshape(-1)
+        t = np.zeros(32, np.uint16)
+        n_out = int(self.lib.oracle_symbol_table(_ptr(w), w.size, _ptr(t)))
+        return t, n_out
+
+    def encode_v4(self, w: np.ndarray) -> np.ndarray:
+        w = np.ascontiguousarray(w, dtype=np.uint16)
+        rows, cols = w.shape
+        nbytes = C.c_uint64(0)
+        _check(self.lib.oracle_encode_v4(_ptr(w), rows, cols, None, 0, C.byref(nbytes)), "encode_v4 size")
+        out = np.zeros(nbytes.value, np.uint8)
+        _check(self.lib.oracle_encode_v4(_ptr(w), rows, cols, _ptr(out), out.size, C.byref(nbytes)), "encode_v4")
+        return out
+
+    def decode_v4(self, blob: np.ndarray) -> np.ndarray:
+        blob = np.ascontiguousarray(blob, dtype=np.uint8)
+        rows, cols = self.shape_of(blob)
+        out = np.zeros((rows, cols), np.uint16)
+        _check(self.lib.oracle_decode_v4(_ptr(blob), blob.size, _ptr(out)), "decode_v4")
+        return out
+
+    def decode_v4_rc(self, blob: np.ndarray) -> int:
+        blob = np.ascontiguousarray(blob, dtype=np.uint8)
+        rows, cols = self.shape_of(blob)
+        out = np.zeros((rows, cols), np.uint16)
+        return int(self.lib.oracle_decode_v4(_ptr(blob), blob.size, _ptr(out)))
 
     def swiglu_f64(self, blob_gate: np.ndarray, blob_up: np.ndarray, x: np.ndarray):
         """Gated MLP input side: g = W_gate x, u = W_up x (FP64 GEMVs of two

@@ -611,6 +611,186 @@ int oracle_decode_v3(const uint8_t *blob, uint64_t bytes, uint16_t *out) {
 }
 
 /* ---------------------------------------------------------------------- */
+/* Container version 4: sign-and-exponent symbol codes.  [W] "What did the
+ * GLM-5.2 experiment actually prove?" describes short fixed codes for the
+ * common sign-and-exponent symbols of a tensor, with rare symbols sent
+ * through an escape stream.  Reading (the plainest one that keeps a 12-bit
+ * rate beside the 7 mantissa bits): the symbol of w is its top 9 bits,
+ * s = w >> 7 (sign and exponent); the tensor's table holds its 31 most
+ * frequent symbols (count descending, ties to the smaller symbol; unused
+ * entries 0xFFFF); code = the symbol's index in the table, or 31 (escape).
+ * The 5-bit code and the mantissa are split like version 1's fields:
+ *     raw byte = (code & 1) << 7 | mantissa          (u8 per weight)
+ *     nibble   = code >> 1                           (two per byte, low first)
+ * so w = table[code] << 7 | (raw & 0x7F) for code < 31.  Escapes, their
+ * row-major order and the per-tile offsets are those of version 1 (tile =
+ * 128 weights of a row).  Container: header (version = 4), then
+ *     table   u16[32]        the 31 symbols and one zero entry
+ *     raw     u8 [rows*cols]
+ *     code    u8 [rows*cols/2]
+ *     esc_off u32[n_tiles + 1]
+ *     esc     u16[n_esc]
+ * each part on a 256-byte boundary. */
+#define ORACLE_SYM_CODES 31u
+#define ORACLE_SYM_ESCAPE 31u
+#define ORACLE_SYM_UNUSED 0xFFFFu
+
+typedef struct {
+    uint64_t rows, cols, n_tiles, n_esc;
+    uint64_t off_table, off_raw, off_code, off_esc_off, off_esc, total;
+} oracle_layout4;
+
+static int layout4_for(uint64_t rows, uint64_t cols, uint64_t n_esc, oracle_layout4 *L) {
+    if (cols == 0 || cols % ORACLE_TILE != 0 || rows == 0) return ORACLE_ERR_SHAPE;
+    if (rows > (UINT64_C(1) << 40) / cols) return ORACLE_ERR_SHAPE;
+    L->rows = rows;
+    L->cols = cols;
+    L->n_tiles = rows * (cols / ORACLE_TILE);
+    L->n_esc = n_esc;
+    L->off_table = pad_to_align(ORACLE_HEADER_USED);
+    L->off_raw = L->off_table + pad_to_align(2 * 32);
+    L->off_code = L->off_raw + pad_to_align(rows * cols);
+    L->off_esc_off = L->off_code + pad_to_align(rows * cols / 2);
+    L->off_esc = L->off_esc_off + pad_to_align(4 * (L->n_tiles + 1));
+    L->total = L->off_esc + pad_to_align(2 * L->n_esc);
+    return ORACLE_OK;
+}
+
+int64_t oracle_container_bytes_v4(uint64_t rows, uint64_t cols, uint64_t n_esc) {
+    oracle_layout4 L;
+    int rc = layout4_for(rows, cols, n_esc, &L);
+    if (rc != ORACLE_OK) return rc;
+    return (int64_t)L.total;
+}
+
+/* The symbol table of a tensor: its 31 most frequent symbols, count
+ * descending, ties to the smaller symbol; table[i] = 0xFFFF past the number
+ * of distinct symbols.  Returns the number of weights outside the table. */
+uint64_t oracle_symbol_table(const uint16_t *w, uint64_t n, uint16_t table[32]) {
+    uint64_t count[512];
+    memset(count, 0, sizeof count);
+    for (uint64_t i = 0; i < n; i++) count[w[i] >> 7]++;
+    uint8_t taken[512];
+    memset(taken, 0, sizeof taken);
+    uint64_t covered = 0;
+    for (uint32_t k = 0; k < 32; k++) table[k] = ORACLE_SYM_UNUSED;
+    for (uint32_t k = 0; k < ORACLE_SYM_CODES; k++) {
+        int best = -1;
+        for (int s = 0; s < 512; s++) {
+            if (taken[s] || count[s] == 0) continue;
+            if (best < 0 || count[s] > count[best]) best = s; /* strictly more: ties keep the smaller */
+        }
+        if (best < 0) break;
+        taken[best] = 1;
+        table[k] = (uint16_t)best;
+        covered += count[best];
+    }
+    table[31] = 0;
+    return n - covered;
+}
+
+static uint32_t symbol_code(const uint16_t table[32], uint16_t w) {
+    const uint16_t s = (uint16_t)(w >> 7);
+    for (uint32_t k = 0; k < ORACLE_SYM_CODES; k++)
+        if (table[k] == s) return k;
+    return ORACLE_SYM_ESCAPE;
+}
+
+/* Encoder, version 4. */
+int oracle_encode_v4(const uint16_t *w, uint64_t rows, uint64_t cols, uint8_t *dst, uint64_t cap,
+                     uint64_t *bytes_out) {
+    if (!w || !bytes_out) return ORACLE_ERR_ARG;
+    oracle_layout4 L;
+    int rc = layout4_for(rows, cols, 0, &L);
+    if (rc != ORACLE_OK) return rc;
+    uint16_t table[32];
+    const uint64_t n_esc = oracle_symbol_table(w, rows * cols, table);
+    if (n_esc > 0xFFFFFFFFull) return ORACLE_ERR_SHAPE; /* esc_off is u32 */
+    layout4_for(rows, cols, n_esc, &L);
+    *bytes_out = L.total;
+    if (!dst) return ORACLE_OK;
+    if (cap < L.total) return ORACLE_ERR_CAPACITY;
+
+    memset(dst, 0, L.total);
+    memcpy(dst, "S12\0", 4);
+    put_u32(dst + 4, 4);
+    put_u64(dst + 8, rows);
+    put_u64(dst + 16, cols);
+    put_u32(dst + 24, ORACLE_TILE);
+    put_u32(dst + 28, 0);
+    put_u64(dst + 32, n_esc);
+    uint8_t *tab = dst + L.off_table, *raw = dst + L.off_raw, *code = dst + L.off_code;
+    uint8_t *off = dst + L.off_esc_off, *esc = dst + L.off_esc;
+    for (uint32_t k = 0; k < 32; k++) {
+        tab[2 * k] = (uint8_t)(table[k] & 0xFF);
+        tab[2 * k + 1] = (uint8_t)(table[k] >> 8);
+    }
+    uint64_t written = 0;
+    for (uint64_t pos = 0; pos < rows * cols; pos++) {
+        if (pos % ORACLE_TILE == 0) put_u32(off + 4 * (pos / ORACLE_TILE), (uint32_t)written);
+        const uint16_t v = w[pos];
+        const uint32_t c = symbol_code(table, v);
+        raw[pos] = (uint8_t)(((c & 1u) << 7) | oracle_bf16_mantissa(v));
+        const uint32_t nib = c >> 1;
+        if (pos % 2 == 0)
+            code[pos / 2] = (uint8_t)nib;
+        else
+            code[pos / 2] |= (uint8_t)(nib << 4);
+        if (c == ORACLE_SYM_ESCAPE) {
+            esc[2 * written] = (uint8_t)(v & 0xFF);
+            esc[2 * written + 1] = (uint8_t)(v >> 8);
+            written++;
+        }
+    }
+    put_u32(off + 4 * L.n_tiles, (uint32_t)written);
+    return ORACLE_OK;
+}
+
+/* Decoder, version 4, with the checks: the table's used entries are valid
+ * 9-bit symbols, no code points at an unused entry, offsets start at 0, end
+ * at n_esc and never decrease, and each tile's escape count equals its
+ * offset span. */
+int oracle_decode_v4(const uint8_t *blob, uint64_t bytes, uint16_t *out) {
+    if (!blob || !out) return ORACLE_ERR_ARG;
+    if (bytes < ORACLE_HEADER_USED || memcmp(blob, "S12\0", 4) != 0) return ORACLE_ERR_CORRUPT;
+    if (get_u32(blob + 4) != 4 || get_u32(blob + 24) != ORACLE_TILE || get_u32(blob + 28) != 0)
+        return ORACLE_ERR_CORRUPT;
+    for (int i = 40; i < 64; i++)
+        if (blob[i] != 0) return ORACLE_ERR_CORRUPT;
+    uint64_t rows = get_u64(blob + 8), cols = get_u64(blob + 16), n_esc = get_u64(blob + 32);
+    oracle_layout4 L;
+    if (layout4_for(rows, cols, n_esc, &L) != ORACLE_OK) return ORACLE_ERR_CORRUPT;
+    if (n_esc > rows * cols || bytes < L.total) return ORACLE_ERR_CORRUPT;
+    const uint8_t *tab = blob + L.off_table, *raw = blob + L.off_raw, *code = blob + L.off_code;
+    const uint8_t *off = blob + L.off_esc_off, *esc = blob + L.off_esc;
+    uint16_t table[32];
+    for (uint32_t k = 0; k < 32; k++) table[k] = get_u16(tab + 2 * k);
+    for (uint32_t k = 0; k < ORACLE_SYM_CODES; k++)
+        if (table[k] != ORACLE_SYM_UNUSED && table[k] > 511) return ORACLE_ERR_CORRUPT;
+    if (get_u32(off) != 0 || get_u32(off + 4 * L.n_tiles) != n_esc) return ORACLE_ERR_CORRUPT;
+    for (uint64_t t = 0; t < L.n_tiles; t++) {
+        const uint64_t lo = get_u32(off + 4 * t), hi = get_u32(off + 4 * (t + 1));
+        if (hi < lo || hi > n_esc) return ORACLE_ERR_CORRUPT;
+        uint64_t k = lo;
+        for (uint32_t i = 0; i < ORACLE_TILE; i++) {
+            const uint64_t pos = t * ORACLE_TILE + i;
+            const uint32_t nib = (pos % 2 == 0) ? (code[pos / 2] & 0x0Fu) : (uint32_t)(code[pos / 2] >> 4);
+            const uint32_t c = (nib << 1) | (uint32_t)(raw[pos] >> 7);
+            if (c < ORACLE_SYM_CODES) {
+                if (table[c] == ORACLE_SYM_UNUSED) return ORACLE_ERR_CORRUPT;
+                out[pos] = (uint16_t)(((uint32_t)table[c] << 7) | (raw[pos] & 0x7Fu));
+            } else {
+                if (k >= hi) return ORACLE_ERR_CORRUPT;
+                out[pos] = get_u16(esc + 2 * k);
+                k++;
+            }
+        }
+        if (k != hi) return ORACLE_ERR_CORRUPT;
+    }
+    return ORACLE_OK;
+}
+
+/* ---------------------------------------------------------------------- */
 /* Dense product in FP64: y[m][n] = sum_k W[n][k] * x[m][k], and the
  * tolerance scale s[m][n] = sum_k |W[n][k] * x[m][k]|.  Every BF16 operand
  * converts exactly; the product of two BF16 values is exact in FP64.  This

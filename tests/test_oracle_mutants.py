@@ -65,6 +65,12 @@ MUTANTS = {
          "(pos % 2 == 1) ? (pair[3 * p + 2] & 0x0Fu) : (uint32_t)(pair[3 * p + 2] >> 4)")],
     "v3_pair_plane_unpadded": [("L->off_base = L->off_pair + pad_to_align(rows * cols / 2 * 3);",
                                 "L->off_base = L->off_pair + rows * cols / 2 * 3;")],
+    "v4_ties_to_larger_symbol": [("if (best < 0 || count[s] > count[best]) best = s;",
+                                  "if (best < 0 || count[s] >= count[best]) best = s;")],
+    "v4_table_of_30_symbols": [("    for (uint32_t k = 0; k < ORACLE_SYM_CODES; k++) {\n        int best = -1;",
+                                "    for (uint32_t k = 0; k + 1 < ORACLE_SYM_CODES; k++) {\n        int best = -1;")],
+    "v4_code_bit_dropped_from_raw": [("raw[pos] = (uint8_t)(((c & 1u) << 7) | oracle_bf16_mantissa(v));",
+                                      "raw[pos] = (uint8_t)oracle_bf16_mantissa(v);")],
     "escape_stored_byte_swapped": [("esc[2 * *written] = (uint8_t)(v & 0xFF);\n            esc[2 * *written + 1] = (uint8_t)(v >> 8);",
                                     "esc[2 * *written] = (uint8_t)(v >> 8);\n            esc[2 * *written + 1] = (uint8_t)(v & 0xFF);")],
 }
@@ -136,6 +142,11 @@ def _battery(o: Oracle):
     pr = b3[256:256 + 16 * 1024 * 3 // 2].reshape(-1, 3)
     assert np.array_equal(pr[:, 2], b1[256 + 16 * 1024:256 + 16 * 1024 + 8192])
     assert np.array_equal(pr[:, 0], b1[256:256 + 16 * 1024:2])
+    # container version 4: the hand-derived golden and a round trip
+    d4 = load_golden("one_tile_v4.json")
+    w4 = np.array([int(x, 16) for x in d4["weights"]], np.uint16).reshape(1, 128)
+    assert np.array_equal(o.encode_v4(w4), golden_expected_bytes(d4))
+    assert np.array_equal(o.decode_v4(o.encode_v4(wv)), wv)
     # gated-MLP activation: textbook values of t * logistic(t)
     e = np.e
     h = o.silu_mul_f64(np.array([1.0, 2.0, 64.0, -64.0, 0.0]), np.array([2.0, 1.0, 3.0, 3.0, 5.0]))
