@@ -116,6 +116,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Para
     const uint32_t stages = sb + 256;
     const uint32_t slots = stages + kStages * kStageB;           // 2 per decode warp
     __shared__ uint32_t s_hist[256];  // histogram mode
+    __shared__ uint32_t s_tab[32];    // version 4: the symbol table
     const long long n_chunks = (p.n_tiles + kChunkTiles - 1) / kChunkTiles;
     const long long c0 = chunk_start(blockIdx.x, n_chunks, gridDim.x), c1 = chunk_start(blockIdx.x + 1, n_chunks, gridDim.x);
     if (threadIdx.x == 0) {
@@ -127,6 +128,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Para
     }
     if (HIST)
         for (int i = threadIdx.x; i < 256; i += kThreads) s_hist[i] = 0;
+    if (V == 4 && threadIdx.x < 32) s_tab[threadIdx.x] = __ldg(static_cast<const uint16_t *>(p.meta) + threadIdx.x);
     __syncthreads();
 
     if (warp == 0) {
@@ -140,7 +142,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Para
             mb = mo = me = 0;
             if (lane < nt) {
                 if (V != 2) {
-                    mb = __ldg(static_cast<const uint8_t *>(p.meta) + t);
+                    mb = V == 4 ? 0u : __ldg(static_cast<const uint8_t *>(p.meta) + t);
                     mo = __ldg(p.off + t);
                 } else {
                     const uint32_t w = __ldg(static_cast<const uint16_t *>(p.meta) + t);
@@ -298,8 +300,40 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Para
                 // last tile: at the chunk's end)
                 hi = lds32(meta + 4 * (kChunkTiles + 1) + 4 * (tl + 1 < nt ? tl + 1 : kChunkTiles));
             }
-            if (base > static_cast<uint32_t>(kMaxBase)) raise_flag(p.err, S12_FLAG_BASE);
-            const uint32_t m0 = escape_nibbles(code.x), m1 = escape_nibbles(code.y);
+            uint32_t m0, m1;
+            uint32_t w[8];
+            if (V == 4) {
+                // code = nibble << 1 | raw bit 7; the weight is table[code] << 7
+                // | mantissa, or an escape (code 31, flagged like a version 1
+                // escape nibble: bit 4j+3 of m0 / m1)
+                m0 = m1 = 0;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const uint32_t rw = j < 4 ? raw.x : j < 8 ? raw.y : j < 12 ? raw.z : raw.w;
+                    const uint32_t r = (rw >> (8 * (j & 3))) & 0xFFu;
+                    const uint32_t nib = ((j < 8 ? code.x : code.y) >> (4 * (j & 7))) & 0xFu;
+                    const uint32_t cd = (nib << 1) | (r >> 7);
+                    uint32_t v = 0;
+                    if (cd == 31u) {
+                        if (j < 8)
+                            m0 |= 8u << (4 * j);
+                        else
+                            m1 |= 8u << (4 * (j - 8));
+                    } else {
+                        const uint32_t sym = s_tab[cd];
+                        if (sym > 511u) raise_flag(p.err, S12_FLAG_BASE);  // an unused table entry
+                        v = ((sym & 0x1FFu) << 7) | (r & 0x7Fu);
+                    }
+                    if (j & 1)
+                        w[j >> 1] |= v << 16;
+                    else
+                        w[j >> 1] = v;
+                }
+            } else {
+                if (base > static_cast<uint32_t>(kMaxBase)) raise_flag(p.err, S12_FLAG_BASE);
+                m0 = escape_nibbles(code.x);
+                m1 = escape_nibbles(code.y);
+            }
             // rank of the lane's first escape within its tile (8 lanes per tile)
             const uint32_t cnt = __popc(m0) + __popc(m1);
             uint32_t incl = cnt;
@@ -309,10 +343,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Para
                 if (piece >= d) incl += v;
             }
             if (active && piece == 7 && incl != hi - lo) raise_flag(p.err, S12_FLAG_ESC_COUNT);
-            uint32_t w[8];
             // with escape nibbles cleared, base + code never carries out of its byte
-            decode16(raw, (m0 | m1) ? make_uint2(clear_escapes(code.x, m0), clear_escapes(code.y, m1)) : code,
-                     base * 0x01010101u, w);
+            if (V != 4)
+                decode16(raw, (m0 | m1) ? make_uint2(clear_escapes(code.x, m0), clear_escapes(code.y, m1)) : code,
+                         base * 0x01010101u, w);
             const uint32_t mine = slot + static_cast<uint32_t>(lane) * 32u;  // tile-major: the output order
             if (active) {
                 asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(mine), "r"(w[0]), "r"(w[1]), "r"(w[2]),
@@ -387,7 +421,9 @@ int run_decode(const s12_view *v, uint16_t *out, unsigned long long *hist, uint3
     dec::Params p;
     p.raw = v->raw;
     p.code = v->code;
-    p.meta = V != 2 ? static_cast<const void *>(v->base) : static_cast<const void *>(v->tmeta);
+    p.meta = V == 4   ? static_cast<const void *>(v->symtab)
+             : V != 2 ? static_cast<const void *>(v->base)
+                      : static_cast<const void *>(v->tmeta);
     p.off = V != 2 ? v->esc_off : v->row_esc;
     p.esc = v->esc;
     p.n_esc = static_cast<uint32_t>(v->n_esc);
@@ -412,6 +448,7 @@ int run_decode(const s12_view *v, uint16_t *out, unsigned long long *hist, uint3
 }  // namespace
 
 int launch_decode(const s12_view *v, uint16_t *out, uint32_t *err, cudaStream_t stream) {
+    if (v->version == 4) return run_decode<4, false>(v, out, nullptr, err, stream);
     if (v->version == 3) return run_decode<3, false>(v, out, nullptr, err, stream);
     return v->version == 1 ? run_decode<1, false>(v, out, nullptr, err, stream)
                            : run_decode<2, false>(v, out, nullptr, err, stream);
@@ -419,6 +456,7 @@ int launch_decode(const s12_view *v, uint16_t *out, uint32_t *err, cudaStream_t 
 
 int launch_stats_hist(const s12_view *v, unsigned long long *hist, cudaStream_t stream) {
     if (cudaMemsetAsync(hist, 0, 256 * sizeof(unsigned long long), stream) != cudaSuccess) return S12_ERR_CUDA;
+    if (v->version == 4) return run_decode<4, true>(v, nullptr, hist, nullptr, stream);
     if (v->version == 3) return run_decode<3, true>(v, nullptr, hist, nullptr, stream);
     return v->version == 1 ? run_decode<1, true>(v, nullptr, hist, nullptr, stream)
                            : run_decode<2, true>(v, nullptr, hist, nullptr, stream);

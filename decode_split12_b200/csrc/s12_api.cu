@@ -29,6 +29,8 @@ int check_view(const s12_view *v) {
         if (!v->code || !v->tmeta || !v->row_esc) return S12_ERR_ARG;
     } else if (v->version == 3) {
         if (!v->base || !v->esc_off) return S12_ERR_ARG;  // raw = the pair plane, no code plane
+    } else if (v->version == 4) {
+        if (!v->code || !v->esc_off || !v->symtab) return S12_ERR_ARG;
     } else {
         return S12_ERR_ARG;
     }
@@ -195,7 +197,7 @@ int s12_open(const void *container, size_t bytes, s12_view *out) {
     if (cudaMemcpy(h, container, sizeof h, cudaMemcpyDeviceToHost) != cudaSuccess) return S12_ERR_CUDA;
     if (std::memcmp(h, "S12\0", 4) != 0) return S12_ERR_CORRUPT;
     const uint32_t version = get_u32(h + 4);
-    if (version < 1 || version > 3 || get_u32(h + 24) != static_cast<uint32_t>(kTile) || get_u32(h + 28) != 0)
+    if (version < 1 || version > 4 || get_u32(h + 24) != static_cast<uint32_t>(kTile) || get_u32(h + 28) != 0)
         return S12_ERR_CORRUPT;
     for (int i = 40; i < 64; ++i)
         if (h[i]) return S12_ERR_CORRUPT;
@@ -219,6 +221,16 @@ int s12_open(const void *container, size_t bytes, s12_view *out) {
         out->raw = c + g.off_raw;
         out->code = c + g.off_code;
         out->base = c + g.off_base;
+        out->esc_off = reinterpret_cast<const uint32_t *>(c + g.off_esc_off);
+        out->esc = reinterpret_cast<const uint16_t *>(c + g.off_esc);
+    } else if (version == 4) {
+        const Geometry4 g = geometry4(rows, cols, n_esc);
+        if (g.total > bytes) return S12_ERR_CORRUPT;
+        out->n_tiles = g.n_tiles;
+        out->container_bytes = g.total;
+        out->symtab = reinterpret_cast<const uint16_t *>(c + g.off_table);
+        out->raw = c + g.off_raw;
+        out->code = c + g.off_code;
         out->esc_off = reinterpret_cast<const uint32_t *>(c + g.off_esc_off);
         out->esc = reinterpret_cast<const uint16_t *>(c + g.off_esc);
     } else if (version == 3) {
@@ -429,7 +441,9 @@ int s12_stats(const s12_view *v, s12_stats_t *out, void *ws, size_t ws_bytes, vo
     out->n_esc = v->n_esc;
     out->container_bytes = v->container_bytes;
     out->payload_bytes = nw + nw / 2;
-    out->header_bytes = v->version == 2 ? v->n_tiles * 2 + 4 * (v->rows + 1) : v->n_tiles * 5;
+    out->header_bytes = v->version == 2   ? v->n_tiles * 2 + 4 * (v->rows + 1)
+                        : v->version == 4 ? 4 * (v->n_tiles + 1) + 64
+                                          : v->n_tiles * 5;
     out->escape_bytes = 2 * v->n_esc;
     out->escape_rate = static_cast<double>(v->n_esc) / static_cast<double>(nw);
     out->bits_per_weight = 8.0 * static_cast<double>(v->container_bytes) / static_cast<double>(nw);

@@ -92,6 +92,29 @@ __host__ __device__ inline Geometry3 geometry3(uint64_t rows, uint64_t cols, uin
     return g;
 }
 
+// Plane offsets of a version 4 container (sign-and-exponent symbol codes):
+// the symbol table u16[32], then raw, code, esc_off and esc as version 1
+// (no base plane).
+struct Geometry4 {
+    uint64_t rows, cols, n_tiles, n_esc;
+    uint64_t off_table, off_raw, off_code, off_esc_off, off_esc, total;
+};
+
+__host__ __device__ inline Geometry4 geometry4(uint64_t rows, uint64_t cols, uint64_t n_esc) {
+    Geometry4 g;
+    g.rows = rows;
+    g.cols = cols;
+    g.n_tiles = rows * (cols / kTile);
+    g.n_esc = n_esc;
+    g.off_table = kHeaderBytes;
+    g.off_raw = g.off_table + kAlign;  // 64 bytes used
+    g.off_code = g.off_raw + align_up(rows * cols, kAlign);
+    g.off_esc_off = g.off_code + align_up(rows * cols / 2, kAlign);
+    g.off_esc = g.off_esc_off + align_up(4 * (g.n_tiles + 1), kAlign);
+    g.total = g.off_esc + align_up(2 * n_esc, kAlign);
+    return g;
+}
+
 // ---------------------------------------------------------------------------
 // Bounded waiting.  Every spin in these kernels gives up after about a second
 // at full clock, sets S12_FLAG_TIMEOUT and lets the caller unwind.

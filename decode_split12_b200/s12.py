@@ -57,6 +57,7 @@ class View(C.Structure):
         ("container_bytes", C.c_uint64), ("container", C.c_void_p), ("raw", C.c_void_p),
         ("code", C.c_void_p), ("base", C.c_void_p), ("esc_off", C.c_void_p), ("esc", C.c_void_p),
         ("version", C.c_uint32), ("reserved", C.c_uint32), ("tmeta", C.c_void_p), ("row_esc", C.c_void_p),
+        ("symtab", C.c_void_p),
     ]
 
 

@@ -81,7 +81,8 @@ extern "C" {
 /* ---- err_flag bits set by kernels ---- */
 #define S12_FLAG_ESC_COUNT 1u   /* a tile's code-15 count != its esc_off span */
 #define S12_FLAG_ESC_RANGE 2u   /* esc_off points outside the escape stream   */
-#define S12_FLAG_BASE 4u        /* a tile base above 241                      */
+#define S12_FLAG_BASE 4u        /* a tile base above 241 (version 4: a code
+                                   of an unused symbol-table entry)           */
 #define S12_FLAG_TIMEOUT 8u     /* a bounded wait inside a kernel gave up     */
 
 #define S12_TILE 128
@@ -99,9 +100,14 @@ extern "C" {
  * deep dive: weights 2i and 2i+1 stored as raw(2i), raw(2i+1),
  * code(2i) | code(2i+1) << 4 in one pair plane of rows*cols*3/2 bytes, then
  * version 1's base, esc_off and esc planes) has `raw` pointing at the pair
- * plane, NULL `code`, and `base`/`esc_off` as version 1.  Decode and stats
- * read all three versions; the fused GEMV and GEMM read versions 1 and 2
- * (S12_ERR_ARG for version 3). */
+ * plane, NULL `code`, and `base`/`esc_off` as version 1.  A version 4
+ * container (sign-and-exponent symbol codes, [W] "What did the GLM-5.2
+ * experiment actually prove?": the tensor's 31 most frequent sign+exponent
+ * symbols, w >> 7, in a table; code = the index or 31 for an escape;
+ * raw = (code & 1) << 7 | mantissa; nibble = code >> 1) has `symtab`, `raw`,
+ * `code` and `esc_off` (tile offsets as version 1) and NULL base.  Decode and
+ * stats read all four versions; the fused GEMV and GEMM read versions 1 and
+ * 2 (S12_ERR_ARG otherwise). */
 typedef struct s12_view {
     uint64_t rows;            /* output features (N)                      */
     uint64_t cols;            /* input features (K), multiple of 128      */
@@ -114,17 +120,18 @@ typedef struct s12_view {
     const uint8_t *base;      /* version 1: u8 [n_tiles]                  */
     const uint32_t *esc_off;  /* version 1: u32[n_tiles+1]                */
     const uint16_t *esc;      /* u16[n_esc]                               */
-    uint32_t version;         /* 1, 2 or 3                                */
+    uint32_t version;         /* 1 .. 4                                   */
     uint32_t reserved;        /* 0                                        */
     const uint16_t *tmeta;    /* version 2: u16[n_tiles], base | count<<8 */
     const uint32_t *row_esc;  /* version 2: u32[rows+1], escapes before r */
+    const uint16_t *symtab;   /* version 4: u16[32], the symbol table     */
 } s12_view;
 
 typedef struct s12_stats_t {
     uint64_t rows, cols, n_tiles, n_esc;
     uint64_t container_bytes; /* everything, padding included            */
     uint64_t payload_bytes;   /* raw + code = 1.5 bytes per weight       */
-    uint64_t header_bytes;    /* v1, v3: 5 per tile; v2: 2 per tile + 4 per row */
+    uint64_t header_bytes;    /* v1, v3: 5 per tile; v2: 2 per tile + 4 per row; v4: 4 per tile + 68 */
     uint64_t escape_bytes;    /* 2 bytes per escape                      */
     double escape_rate;       /* n_esc / (rows*cols)                     */
     double bits_per_weight;   /* 8 * container_bytes / (rows*cols)       */
@@ -177,7 +184,7 @@ int s12_encode(const uint16_t *w, int64_t rows, int64_t cols, void *dst, size_t 
 /* Follows: the container layout above, which restates [M] section 1 (the
  * BF16 bit fields) and [T] key points (tile base, escape stream).
  * Validate the 64-byte header of a container (device, `bytes` long, version
- * 1, 2 or 3) and fill *out with its shape, version and plane pointers.  Copies
+ * 1 to 4) and fill *out with its shape, version and plane pointers.  Copies
  * the header to the host and so SYNCHRONISES (the legacy default stream).
  * S12_ERR_CORRUPT on a bad magic, version, tile size, flags, shape or a size
  * above `bytes`. */

@@ -318,3 +318,56 @@ def test_v3_decode_full_size_and_stats(s12, oracle):
         s12.s12_gemv(v3, to_dev(wl.activations(1, 1152, 0)))
     with pytest.raises(s12.S12Error):
         s12.s12_gemm_skinny(v3, to_dev(wl.activations(16, 1152, 0)))
+
+
+# ---------------------------------------------------------------------------
+# container version 4 (sign-and-exponent symbol codes), built by the oracle
+
+@pytest.mark.parametrize("order", ["natural", "shuffled"])
+def test_v4_decode_all_patterns(s12, oracle, order):
+    """All 65,536 BF16 patterns as a version 4 container (a tensor table of
+    31 sign+exponent symbols; [W] "What did the GLM-5.2 experiment actually
+    prove?"): the GPU decode gives every bit back."""
+    w = _all_patterns(order)
+    view = s12.s12_open(blob_to_dev(oracle.encode_v4(w)))
+    assert view.version == 4
+    flag = new_flag()
+    out = s12.s12_decode(view, err_flag=flag)
+    torch.cuda.synchronize()
+    assert np.array_equal(from_dev_u16(out), w)
+    assert int(flag.item()) == 0
+
+
+@pytest.mark.parametrize("shape", [(1, 128), (3, 384), (67, 384), (300, 1152), (5, 14336)])
+@pytest.mark.parametrize("kind", ["student", "stress"])
+def test_v4_decode_shapes(s12, oracle, shape, kind):
+    r, c = shape
+    w = wl.student_t_scaled(r, c, r + c) if kind == "student" else wl.escape_stress(0.05, r + 2 * c, r, c)[0]
+    view = s12.s12_open(blob_to_dev(oracle.encode_v4(w)))
+    flag = new_flag()
+    out = s12.s12_decode(view, err_flag=flag)
+    torch.cuda.synchronize()
+    assert np.array_equal(from_dev_u16(out), w)
+    assert int(flag.item()) == 0
+
+
+def test_v4_decode_full_size_and_stats(s12, oracle):
+    """The 8B-style gate projection (14336 x 4096) as a version 4 container:
+    bit-exact; its statistics equal the oracle's of the version 1 container;
+    the fused products refuse version 4."""
+    w = wl.student_t_scaled(14336, 4096, 0, 4)
+    view = s12.s12_open(blob_to_dev(oracle.encode_v4(w)))
+    flag = new_flag()
+    out = s12.s12_decode(view, err_flag=flag)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), to_dev(w))
+    assert int(flag.item()) == 0
+    small = wl.student_t_scaled(300, 1152, 7)
+    ref = oracle.stats(oracle.encode(small))
+    v4 = s12.s12_open(blob_to_dev(oracle.encode_v4(small)))
+    st = s12.s12_stats(v4)
+    assert st["exp_hist"] == [int(h) for h in ref["exp_hist"]]
+    with pytest.raises(s12.S12Error):
+        s12.s12_gemv(v4, to_dev(wl.activations(1, 1152, 0)))
+    with pytest.raises(s12.S12Error):
+        s12.s12_gemm_skinny(v4, to_dev(wl.activations(16, 1152, 0)))
