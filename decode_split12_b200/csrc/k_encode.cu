@@ -374,8 +374,10 @@ int launch_encode(const uint16_t *w, int64_t rows, int64_t cols, void *dst, size
     const uint64_t n_groups = (n_tiles + kTilesPerWarp - 1) / kTilesPerWarp;
     if (ws_bytes < encode_ws_bytes(rows, cols)) return S12_ERR_CAPACITY;
     const Geometry g0 = geometry(R, C, 0);
-    if (dst && dst_cap < g0.total) return S12_ERR_CAPACITY;
-    uint8_t *d = static_cast<uint8_t *>(dst);
+    // a destination smaller than the escape-free size is not written: the
+    // call then works as a size query and reports S12_ERR_CAPACITY
+    const bool too_small = dst && dst_cap < g0.total;
+    uint8_t *d = too_small ? nullptr : static_cast<uint8_t *>(dst);
 
     EncodeParams p;
     p.w = w;
@@ -409,7 +411,7 @@ int launch_encode(const uint16_t *w, int64_t rows, int64_t cols, void *dst, size
     if (cudaStreamSynchronize(stream) != cudaSuccess) return S12_ERR_CUDA;
     const Geometry g = geometry(R, C, n_esc);
     *bytes_out = static_cast<size_t>(g.total);
-    if (d && dst_cap < g.total) return S12_ERR_CAPACITY;
+    if (too_small || (d && dst_cap < g.total)) return S12_ERR_CAPACITY;
     return S12_OK;
 }
 

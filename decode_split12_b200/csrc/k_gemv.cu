@@ -28,22 +28,25 @@
 // on B200 with the copies alone, that streams at the copy bandwidth, while
 // one tile per copy (128- and 64-byte row pieces) stays near 65 % of it.
 //
-// Per-tile metadata.  The four lanes of a quad share a row, so each lane
-// fetches one metadata word of its two rows per stage and the quad exchanges
-// them with shuffles: for a version 1 container the bases and escape-offset
-// ends of the stage's two tiles, for version 2 the two (base | count) words.
-// The escape stream is walked with a running offset per row, so a tile with
-// no escapes (nearly all of them) costs no offset arithmetic, and the
-// decision "does this block hold an escape" comes from the metadata, not from
+// Per-tile metadata.  Each lane loads, a stage ahead, the metadata of its
+// tile for its two rows, as loaded words (arithmetic on them at load time
+// would make the warp wait there): for a version 1 container the base and
+// the tile's escape span from esc_off, for version 2 the stage's two
+// (base | count) words and, at a row group's first stage, the row's escape
+// offset, from which the spans follow as a running offset per row.  The
+// decision "does this stage hold an escape" comes from the spans, not from
 // scanning the code nibbles (which the checked variant still does).
 //
-// Escapes.  A block whose tiles all have empty escape spans takes the straight
-// path.  Otherwise each affected row ranks its escapes across the quad with
-// shuffles, and each half that holds one is patched through a 32-byte
-// per-lane shared scratch: the decoded words are stored, every escaped weight
-// is overwritten by one 16-bit store of its exact value, and the words are
-// read back.  With a tile base of 241, base + 15 would carry into the next
-// byte, so such halves are decoded again with the escape nibbles cleared.
+// Escapes.  A stage whose tile rows all have empty escape spans takes the
+// straight path, one loop-free body.  Otherwise the stage goes through one
+// compact loop over its chunks: the first half of a tile row finds its
+// first escape at the span's start, the second half counts back from the
+// span's end (its escapes are the row's last), and each chunk with an escape
+// is patched through a 32-byte per-lane shared scratch: the decoded words
+// are stored, every escaped weight is overwritten by one 16-bit store of its
+// exact value, and the words are read back.  With a tile base of 241,
+// base + 15 would carry into the next byte, so such chunks are decoded again
+// with the escape nibbles cleared.
 //
 // Work split (stream-K).  Blocks are numbered row-group-major (16-row group,
 // then tile) across all matrices of the call and dealt to all warps of the

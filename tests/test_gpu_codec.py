@@ -198,10 +198,20 @@ def test_size_query_and_capacity(s12, oracle):
     assert lib.s12_encode(C.c_void_p(wd.data_ptr()), 8, 256, None, 0, C.byref(n), C.c_void_p(ws.data_ptr()),
                           ws.numel(), st) == 0
     assert n.value == oracle.encode_size(w)
-    small = torch.empty(n.value - 256, dtype=torch.uint8, device="cuda")
-    rc = lib.s12_encode(C.c_void_p(wd.data_ptr()), 8, 256, C.c_void_p(small.data_ptr()), small.numel(),
-                        C.byref(n), C.c_void_p(ws.data_ptr()), ws.numel(), st)
-    assert rc == s12.S12_ERR_CAPACITY
+    exact = n.value
+    # too small for the escapes only, and smaller than the escape-free size:
+    # both report S12_ERR_CAPACITY with the size needed
+    for cap in (exact - 256, 512):
+        small = torch.zeros(cap, dtype=torch.uint8, device="cuda")
+        n2 = C.c_size_t(0)
+        rc = lib.s12_encode(C.c_void_p(wd.data_ptr()), 8, 256, C.c_void_p(small.data_ptr()), small.numel(),
+                            C.byref(n2), C.c_void_p(ws.data_ptr()), ws.numel(), st)
+        assert rc == s12.S12_ERR_CAPACITY and n2.value == exact
+    # and a destination of the reported size gets the oracle's container
+    blob = torch.zeros(exact, dtype=torch.uint8, device="cuda")
+    assert lib.s12_encode(C.c_void_p(wd.data_ptr()), 8, 256, C.c_void_p(blob.data_ptr()), exact, C.byref(n),
+                          C.c_void_p(ws.data_ptr()), ws.numel(), st) == 0
+    assert np.array_equal(blob.cpu().numpy(), oracle.encode(w))
 
 
 # ---------------------------------------------------------------------------
