@@ -10,7 +10,14 @@ BF16 GB/s = 2 bytes x weights / time, with the fraction of the measured HBM
 copy bandwidth achieved on the compressed bytes actually moved.
 
     python bench.py [--gpus N --steps K --warmup W] [--impl reference]
-                    [--workload llama8b|single|escape|mlp70b|stack]
+                    [--workload llama8b|single] [--batch B]
+                    [--no-cpu-baseline] [--no-gemm] [--no-decode] [--no-stack]
+
+The line's roofline.comparisons carry the uncompressed BF16 GEMV on the same
+layer, the 4096 x 4096 single tensor, the layer from version 2 containers
+and the encoder; `extra` the other batches, launch groupings, the SwiGLU
+epilogue, the skinny GEMM, the standalone decode, the 32-layer stack (also
+as an activation chain) and the MoE block.
 
 Several GPUs run independent replicas (the path does not shard): every
 rank times its own copy and rank 0 reports the sum of work over the max
