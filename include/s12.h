@@ -277,7 +277,7 @@ int s12_gemv_multi(const s12_view *views, int count, const uint16_t *const *x, i
  * The warp-level product gives each lane rows r and r + 8 of a 16-row group,
  * which here are gate row f and up row f: the activation is applied where
  * the sums are stored ([W] "What does 'lossless' mean for LLM weights?":
- * decode and use the weights at once; the epilogue is this build's own). */
+ * decode and use the weights at once; the epilogue is this library's own). */
 int s12_gemv_swiglu(const s12_view *v, const uint16_t *x, int B, uint16_t *h, void *ws, size_t ws_bytes,
                     uint32_t *err_flag, void *stream);
 

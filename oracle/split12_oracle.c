@@ -485,7 +485,7 @@ int oracle_decode_v2(const uint8_t *blob, uint64_t bytes, uint16_t *out) {
 /* ---------------------------------------------------------------------- */
 /* Container version 3: packed 24-bit pairs.  [T] technical deep dive says
  * the 12-bit representation is packed into 3-byte words, two weights per
- * word.  Reading (the plainest one with this build's 12-bit split): weights
+ * word.  Reading (the plainest one with the 12-bit split above): weights
  * 2i and 2i+1 (row-major, always in the same tile) form pair i, stored as
  * three consecutive bytes
  *     byte 3i     raw(w[2i])
