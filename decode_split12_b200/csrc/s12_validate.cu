@@ -224,3 +224,75 @@ extern "C" int s12_from_v2_host(const void *v2, size_t v2_bytes, void *dst, size
     wr32(d + g.off_esc_off + 4 * g.n_tiles, static_cast<uint32_t>(n_esc));
     return S12_OK;
 }
+
+// ---------------------------------------------------------------------------
+// Container version 3 (packed 24-bit pairs) as a storage format: version 1
+// with the raw and code planes regrouped into one pair plane (weights 2i and
+// 2i+1 as raw, raw, code | code << 4; "GPU 友善 12 位無損 BF16 壓縮格式",
+// technical deep dive: two 12-bit weights per 3-byte word).  The metadata
+// and escape planes are version 1's, byte for byte.
+
+extern "C" int s12_to_v3_host(const void *v1, size_t v1_bytes, void *dst, size_t dst_cap, size_t *bytes_out) {
+    if (!v1 || !bytes_out) return S12_ERR_ARG;
+    s12_report rep;
+    const int rc = s12_validate_host(v1, v1_bytes, &rep);
+    if (rc != S12_OK) return rc;
+    const uint8_t *c = static_cast<const uint8_t *>(v1);
+    const Geometry g = geometry(rd64(c + 8), rd64(c + 16), rd64(c + 32));
+    const Geometry3 g3 = geometry3(g.rows, g.cols, g.n_esc);
+    *bytes_out = g3.total;
+    if (!dst) return S12_OK;
+    if (dst_cap < g3.total) return S12_ERR_CAPACITY;
+    uint8_t *d = static_cast<uint8_t *>(dst);
+    std::memset(d, 0, g3.total);
+    std::memcpy(d, c, 64);
+    wr32(d + 4, 3);
+    const uint8_t *raw = c + g.off_raw, *code = c + g.off_code;
+    uint8_t *pair = d + g3.off_pair;
+    for (uint64_t i = 0; i < g.rows * g.cols / 2; ++i) {
+        pair[3 * i] = raw[2 * i];
+        pair[3 * i + 1] = raw[2 * i + 1];
+        pair[3 * i + 2] = code[i];
+    }
+    std::memcpy(d + g3.off_base, c + g.off_base, g.n_tiles);
+    std::memcpy(d + g3.off_esc_off, c + g.off_esc_off, 4 * (g.n_tiles + 1));
+    std::memcpy(d + g3.off_esc, c + g.off_esc, 2 * g.n_esc);
+    return S12_OK;
+}
+
+extern "C" int s12_from_v3_host(const void *v3, size_t v3_bytes, void *dst, size_t dst_cap, size_t *bytes_out) {
+    if (!v3 || !bytes_out) return S12_ERR_ARG;
+    const uint8_t *c = static_cast<const uint8_t *>(v3);
+    if (v3_bytes < kHeaderBytes || std::memcmp(c, "S12\0", 4) != 0 || rd32(c + 4) != 3 ||
+        rd32(c + 24) != static_cast<uint32_t>(kTile) || rd32(c + 28) != 0)
+        return S12_ERR_CORRUPT;
+    for (int i = 40; i < 64; ++i)
+        if (c[i]) return S12_ERR_CORRUPT;
+    const uint64_t rows = rd64(c + 8), cols = rd64(c + 16), n_esc = rd64(c + 32);
+    if (rows == 0 || cols == 0 || cols % kTile || rows >= (uint64_t(1) << 32) || cols >= (uint64_t(1) << 32) ||
+        rows * cols >= (uint64_t(1) << 32) || n_esc > rows * cols)
+        return S12_ERR_CORRUPT;
+    const Geometry3 g3 = geometry3(rows, cols, n_esc);
+    if (g3.total > v3_bytes) return S12_ERR_CORRUPT;
+    const Geometry g = geometry(rows, cols, n_esc);
+    *bytes_out = g.total;
+    if (!dst) return S12_OK;
+    if (dst_cap < g.total) return S12_ERR_CAPACITY;
+    uint8_t *d = static_cast<uint8_t *>(dst);
+    std::memset(d, 0, g.total);
+    std::memcpy(d, c, 64);
+    wr32(d + 4, 1);
+    const uint8_t *pair = c + g3.off_pair;
+    for (uint64_t i = 0; i < rows * cols / 2; ++i) {
+        d[g.off_raw + 2 * i] = pair[3 * i];
+        d[g.off_raw + 2 * i + 1] = pair[3 * i + 1];
+        d[g.off_code + i] = pair[3 * i + 2];
+    }
+    std::memcpy(d + g.off_base, c + g3.off_base, g.n_tiles);
+    std::memcpy(d + g.off_esc_off, c + g3.off_esc_off, 4 * (g.n_tiles + 1));
+    std::memcpy(d + g.off_esc, c + g3.off_esc, 2 * n_esc);
+    // the result must be a valid version 1 container (offsets, counts, bases)
+    s12_report rep;
+    const int rc = s12_validate_host(d, g.total, &rep);
+    return rc == S12_OK ? S12_OK : S12_ERR_CORRUPT;
+}

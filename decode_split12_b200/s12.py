@@ -39,7 +39,8 @@ EXPORTED = (
     "s12_gemv_noalloc", "s12_gemv_swiglu", "s12_gemv_bf16", "s12_gemm_ws_bytes", "s12_gemm_skinny",
     "s12_gemm_skinny_bf16", "s12_gemm_multi_ws_bytes",
     "s12_gemm_skinny_multi", "s12_validate_host", "s12_plane_hashes_host", "s12_fnv1a64",
-    "s12_to_v2_host", "s12_from_v2_host", "s12_load_bf16", "s12_stats_ws_bytes",
+    "s12_to_v2_host", "s12_from_v2_host", "s12_to_v3_host", "s12_from_v3_host", "s12_load_bf16",
+    "s12_stats_ws_bytes",
     "s12_stats", "s12_bf16_gemv",
 )
 
@@ -122,7 +123,7 @@ def _lib() -> C.CDLL:
         lib.s12_validate_host.restype = C.c_int
         lib.s12_plane_hashes_host.argtypes = [_P, _SZ, C.POINTER(C.c_uint64)]
         lib.s12_plane_hashes_host.restype = C.c_int
-        for fn in ("s12_to_v2_host", "s12_from_v2_host"):
+        for fn in ("s12_to_v2_host", "s12_from_v2_host", "s12_to_v3_host", "s12_from_v3_host"):
             getattr(lib, fn).argtypes = [_P, _SZ, _P, _SZ, C.POINTER(_SZ)]
             getattr(lib, fn).restype = C.c_int
         lib.s12_load_bf16.argtypes = [_P, _SZ, _P, _P, C.c_uint64, C.c_uint64, _P, _SZ, _P, _P,
@@ -542,6 +543,17 @@ def s12_load_bf16(container, rows: int, cols: int, dev_container, dev_out, dev_e
 def to_v2_host(container) -> np.ndarray:
     """A version 1 container (host array or tensor) as the compact version 2."""
     return _convert("s12_to_v2_host", container)
+
+
+def to_v3_host(container) -> np.ndarray:
+    """A version 1 container (host array or tensor) as version 3 (packed
+    24-bit pairs)."""
+    return _convert("s12_to_v3_host", container)
+
+
+def from_v3_host(container) -> np.ndarray:
+    """A version 3 container back to version 1."""
+    return _convert("s12_from_v3_host", container)
 
 
 def from_v2_host(container) -> np.ndarray:

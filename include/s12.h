@@ -488,6 +488,17 @@ int s12_load_bf16(const void *container, size_t bytes, const uint64_t *expected_
 int s12_to_v2_host(const void *v1, size_t v1_bytes, void *dst, size_t dst_cap, size_t *bytes_out);
 int s12_from_v2_host(const void *v2, size_t v2_bytes, void *dst, size_t dst_cap, size_t *bytes_out);
 
+/* Follows: [T] technical deep dive (the 12-bit representation packed into
+ * 3-byte words, two weights per word).
+ * Container version 3 (packed 24-bit pairs) as a storage format, converted
+ * in HOST memory like version 2 (snprintf-style; S12_ERR_CAPACITY,
+ * S12_ERR_CORRUPT as there): version 1's raw and code planes regrouped into
+ * one pair plane, the base, esc_off and esc planes byte for byte.  A
+ * version 1 source must pass s12_validate_host; converting back gives it
+ * byte for byte, and the result must pass s12_validate_host. */
+int s12_to_v3_host(const void *v1, size_t v1_bytes, void *dst, size_t dst_cap, size_t *bytes_out);
+int s12_from_v3_host(const void *v3, size_t v3_bytes, void *dst, size_t dst_cap, size_t *bytes_out);
+
 /* ---- uncompressed baseline ---- */
 
 /* Follows: the plain matrix-vector product that [W] "What does 'lossless'

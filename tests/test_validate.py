@@ -192,3 +192,55 @@ def test_v2_conversion_of_the_golden_container():
         v2[off:off + chunk.size] = chunk
     assert np.array_equal(s12.to_v2_host(v1), v2)
     assert np.array_equal(s12.from_v2_host(v2), v1)
+
+
+# ---------------------------------------------------------------------------
+# container version 3 (packed 24-bit pairs) as a storage format
+
+@pytest.mark.parametrize("shape,kind", [((1, 128), "normal"), ((37, 640), "normal"), ((64, 1024), "stress"),
+                                        ((16, 4096), "student")])
+def test_v3_conversion_matches_oracle(oracle, shape, kind):
+    """The library's host conversion to version 3 equals the oracle's
+    version 3 encoder byte for byte, and converting back gives the version
+    1 container byte for byte."""
+    r, c = shape
+    if kind == "stress":
+        w, _ = wl.escape_stress(0.02, 2, r, c)
+    elif kind == "student":
+        w = wl.student_t_scaled(r, c, 3)
+    else:
+        w = wl.normal_with_outliers(r, c, 0.02, 0.01, 2 * r + c)
+    v1 = oracle.encode(w)
+    v3 = s12.to_v3_host(v1)
+    assert np.array_equal(v3, oracle.encode_v3(w))
+    assert np.array_equal(s12.from_v3_host(v3), v1)
+
+
+def test_v3_conversion_of_the_golden_container():
+    from conftest import golden_expected_bytes, load_golden
+    g1, g3 = load_golden("two_tiles.json"), load_golden("two_tiles_v3.json")
+    v1 = golden_expected_bytes(g1)
+    v3 = v1.copy()
+    for a, b in g3["clear"]:
+        v3[a:b] = 0
+    for item in g3["patch"]:
+        chunk = np.frombuffer(bytes.fromhex(item[1]) * (item[2] if len(item) > 2 else 1), np.uint8)
+        v3[item[0]:item[0] + chunk.size] = chunk
+    assert np.array_equal(s12.to_v3_host(v1), v3)
+    assert np.array_equal(s12.from_v3_host(v3), v1)
+
+
+def test_v3_conversion_refuses_corrupt_sources(oracle):
+    w, _ = wl.escape_stress(0.05, 5, 16, 1024)
+    v3 = oracle.encode_v3(w)
+    pair0 = 256
+    codes = v3[pair0 + 2:pair0 + 16 * 1024 * 3 // 2:3]
+    k = int(np.flatnonzero((codes & 0x0F) != 0x0F)[3])
+    bad = v3.copy()
+    bad[pair0 + 3 * k + 2] |= 0x0F          # a code turned into an escape: the tile's count no longer matches
+    with pytest.raises(s12.S12Error):
+        s12.from_v3_host(bad)
+    with pytest.raises(s12.S12Error):
+        s12.from_v3_host(oracle.encode(w))  # a version 1 container is not version 3
+    with pytest.raises(s12.S12Error):
+        s12.to_v3_host(v3)                  # nor is a version 3 one version 1
