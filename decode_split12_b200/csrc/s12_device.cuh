@@ -216,69 +216,4 @@ __device__ __forceinline__ uint32_t clear_escapes(uint32_t C, uint32_t m) {
     return C & ~(m | (m >> 1) | (m >> 2) | (m >> 3));
 }
 
-// Replace the weights flagged in (m0, m1) by consecutive escape-stream
-// values starting at index `first`; `limit` is one past the last index this
-// tile may read (tile end, clamped to the stream).  Out-of-range reads are
-// skipped and flagged.
-// If `staged` is set, escapes [stage_lo, stage_hi) are also in shared memory
-// at `esc_smem` (element stage_lo first) and are read from there.
-__device__ __forceinline__ void patch_escapes(uint32_t out[8], uint32_t m0, uint32_t m1, uint64_t first,
-                                              uint64_t limit, const uint16_t *__restrict__ esc, uint32_t *err,
-                                              const uint16_t *esc_smem = nullptr, uint64_t stage_lo = 0,
-                                              uint64_t stage_hi = 0) {
-    uint64_t idx = first;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-        const uint32_t m = (j < 8) ? m0 : m1;
-        if (m & (8u << (4 * (j & 7)))) {
-            uint32_t v = 0;
-            if (idx < limit) {
-                if (esc_smem && idx >= stage_lo && idx < stage_hi)
-                    v = esc_smem[idx - stage_lo];
-                else
-                    v = __ldg(esc + idx);
-            } else {
-                raise_flag(err, S12_FLAG_ESC_RANGE);
-            }
-            ++idx;
-            if (j & 1)
-                out[j >> 1] = (out[j >> 1] & 0x0000FFFFu) | (v << 16);
-            else
-                out[j >> 1] = (out[j >> 1] & 0xFFFF0000u) | v;
-        }
-    }
-}
-
-// Warp-collective escape fix-up for one 16-weight chunk per lane (kept out
-// of line: it is the rare path, and inlining it bloats the hot loops).  The warp
-// covers up to four tiles, eight lanes per tile.  `lo`/`hi` are esc_off[t]
-// and esc_off[t+1] of the lane's tile (read by every lane).  Must be called
-// by all 32 lanes (inactive lanes pass m0 = m1 = 0).  Re-decodes the chunk
-// with escape nibbles cleared and patches the escaped weights; checks each
-// tile's code-15 count against its offsets.
-static __device__ __noinline__ void fix_escapes(uint32_t out[8], uint4 raw, uint2 code, uint32_t B4, uint32_t m0,
-                                            uint32_t m1, uint32_t lo, uint32_t hi, bool active, uint64_t n_esc,
-                                            const uint16_t *__restrict__ esc, uint32_t *err,
-                                            const uint16_t *esc_smem = nullptr, uint64_t stage_lo = 0,
-                                            uint64_t stage_hi = 0) {
-    const int lane = threadIdx.x & 31;
-    const uint32_t cnt = __popc(m0) + __popc(m1);
-    uint32_t incl = cnt;
-#pragma unroll
-    for (int d = 1; d < 8; d <<= 1) {
-        const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, d, 8);
-        if ((lane & 7) >= d) incl += v;
-    }
-    const uint32_t total = __shfl_sync(0xFFFFFFFFu, incl, 7, 8);
-    if (!active) return;
-    if ((lane & 7) == 0 && hi - lo != total) raise_flag(err, S12_FLAG_ESC_COUNT);
-    if (cnt == 0) return;
-    uint2 c2 = make_uint2(clear_escapes(code.x, m0), clear_escapes(code.y, m1));
-    decode16(raw, c2, B4, out);
-    uint64_t limit = hi < n_esc ? hi : n_esc;
-    if (lo > hi) limit = 0;
-    patch_escapes(out, m0, m1, static_cast<uint64_t>(lo) + (incl - cnt), limit, esc, err, esc_smem, stage_lo,
-                  stage_hi);
-}
-
 }  // namespace s12
